@@ -1,0 +1,336 @@
+// Host side of the C ABI declared in include/ola.h: argument validation, buffer ownership,
+// kernel dispatch, the sticky device error word and the host-buffer entry point.
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+
+#include "ola_device.cuh"
+
+namespace ola {
+cudaError_t launch_prefill(int R, int H, int d_k, int d_v, int P, int in_dtype, const void* k,
+                           const void* v, const float* g, const float* beta, float* S_out,
+                           cudaStream_t stream);
+cudaError_t launch_fullstate(const StepArgs& a, int in_dtype, cudaStream_t stream);
+cudaError_t launch_replay_simt(const StepArgs& a, int in_dtype, cudaStream_t stream);
+size_t replay_simt_smem(int d_k, int d_v, int T_max);
+cudaError_t launch_replay_tc(const StepArgs& a, const CUtensorMap& mhi, const CUtensorMap& mlo,
+                             cudaStream_t stream);
+size_t replay_tc_smem(int d_k, int d_v, int B, int T_max);
+bool make_state_map(CUtensorMap* map, const void* base, int RH, int d_k, int d_v);
+cudaError_t launch_split_state(const float* S, void* hi, void* lo, int RH, int d_k, int d_v,
+                               cudaStream_t stream);
+}  // namespace ola
+
+using namespace ola;
+
+struct ola_ctx {
+  ola_geometry g;
+  int device;
+  int t;
+  int sticky;
+  float* S = nullptr;
+  void* S_hi = nullptr;
+  void* S_lo = nullptr;
+  float* W = nullptr;
+  void* Kr = nullptr;
+  float* A = nullptr;
+  int* C = nullptr;
+  float* FS[2] = {nullptr, nullptr};
+  int* err = nullptr;
+  CUtensorMap m_hi, m_lo;
+  // staging buffers of ola_step_host (allocated on first use)
+  void* st[7] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  cudaStream_t last_stream = nullptr;
+};
+
+namespace {
+
+bool pow2_width(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
+bool tc_width(int d) { return d == 64 || d == 128 || d == 256; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+ola_status validate(const ola_geometry* g) {
+  if (!g) return OLA_ERR_INVALID_ARG;
+  if (g->R < 1 || g->H < 1 || g->B < 1 || g->T_max < 1) return OLA_ERR_INVALID_ARG;
+  if (g->in_dtype != OLA_F32 && g->in_dtype != OLA_BF16) return OLA_ERR_INVALID_ARG;
+  if (g->path != OLA_PATH_REPLAY && g->path != OLA_PATH_FULLSTATE) return OLA_ERR_INVALID_ARG;
+  if (g->math != OLA_MATH_FP32 && g->math != OLA_MATH_TENSOR) return OLA_ERR_INVALID_ARG;
+  if (!pow2_width(g->d_k) || !pow2_width(g->d_v)) return OLA_ERR_UNSUPPORTED;
+  if (g->B > 4096 || g->T_max > 32) return OLA_ERR_UNSUPPORTED;
+  if (int64_t(g->R) * g->H * g->B > (int64_t(1) << 30)) return OLA_ERR_UNSUPPORTED;
+  if (g->math == OLA_MATH_TENSOR) {
+    if (g->path != OLA_PATH_REPLAY || g->in_dtype != OLA_BF16) return OLA_ERR_UNSUPPORTED;
+    if (!tc_width(g->d_k) || !tc_width(g->d_v) || g->B < 16) return OLA_ERR_UNSUPPORTED;
+  }
+  return OLA_OK;
+}
+
+struct Sizes {
+  size_t S, S_split, W, Kr, A, C, FS, err;
+  size_t total() const { return S + 2 * S_split + W + Kr + A + C + 2 * FS + err; }
+};
+
+Sizes sizes_of(const ola_geometry* g) {
+  Sizes z{};
+  const size_t R = g->R, H = g->H, B = g->B, T = g->T_max, dk = g->d_k, dv = g->d_v;
+  const size_t e = g->in_dtype == OLA_BF16 ? 2 : 4;
+  z.S = R * H * dv * dk * 4;
+  z.S_split = g->math == OLA_MATH_TENSOR ? R * H * ((dv + 127) / 128 * 128) * dk * 2 : 0;
+  const bool rep = g->path == OLA_PATH_REPLAY;
+  z.W = rep ? T * R * H * B * dv * 4 : 0;
+  z.Kr = rep ? T * R * H * B * dk * e : 0;
+  z.A = rep ? T * R * H * B * 4 : 0;
+  z.C = T * R * B * T * 4;
+  z.FS = rep ? 0 : R * H * B * dv * dk * 4;
+  z.err = 16;
+  return z;
+}
+
+ola_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return OLA_OK;
+  cudaGetLastError();  // clear a non-sticky error
+  return e == cudaErrorMemoryAllocation ? OLA_ERR_OOM : OLA_ERR_CUDA;
+}
+
+template <typename T>
+cudaError_t dev_alloc(T** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) return cudaSuccess;
+  void* q = nullptr;
+  cudaError_t e = cudaMalloc(&q, bytes);
+  if (e == cudaSuccess) *p = static_cast<T*>(q);
+  return e;
+}
+
+void free_all(ola_ctx* h) {
+  void* ptrs[] = {h->S, h->S_hi, h->S_lo, h->W, h->Kr, h->A, h->C, h->FS[0], h->FS[1], h->err};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  for (void* p : h->st)
+    if (p) cudaFree(p);
+}
+
+StepArgs make_args(ola_ctx* h, const void* q, const void* k, const void* v, const float* g,
+                   const float* beta, const int32_t* parent, float* out_o) {
+  StepArgs a;
+  a.R = h->g.R;
+  a.H = h->g.H;
+  a.d_k = h->g.d_k;
+  a.d_v = h->g.d_v;
+  a.B = h->g.B;
+  a.T_max = h->g.T_max;
+  a.t = h->t + 1;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g = g;
+  a.beta = beta;
+  a.parent = parent;
+  a.o = out_o;
+  a.S = h->S;
+  a.W = h->W;
+  a.Kr = h->Kr;
+  a.A = h->A;
+  a.C = h->C;
+  a.FS_prev = h->FS[(a.t + 1) & 1];   // states of step t-1 (unused at t = 1)
+  a.FS_cur = h->FS[a.t & 1];
+  a.err = h->err;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t ola_version(void) { return (1 << 16) | 0; }
+
+const char* ola_strerror(ola_status s) {
+  switch (s) {
+    case OLA_OK: return "ok";
+    case OLA_ERR_INVALID_ARG: return "invalid argument";
+    case OLA_ERR_UNSUPPORTED: return "unsupported geometry or device";
+    case OLA_ERR_CAPACITY: return "step capacity T_max exhausted";
+    case OLA_ERR_BAD_PARENT: return "parent index out of range";
+    case OLA_ERR_OOM: return "device out of memory";
+    case OLA_ERR_CUDA: return "CUDA runtime error";
+    case OLA_ERR_TIMEOUT: return "bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+ola_status ola_workspace_bytes(const ola_geometry* geom, uint64_t* out_bytes) {
+  if (!out_bytes) return OLA_ERR_INVALID_ARG;
+  ola_status s = validate(geom);
+  if (s != OLA_OK) return s;
+  *out_bytes = sizes_of(geom).total();
+  return OLA_OK;
+}
+
+ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream,
+                      ola_handle* out) {
+  if (!out) return OLA_ERR_INVALID_ARG;
+  *out = nullptr;
+  ola_status s = validate(geom);
+  if (s != OLA_OK) return s;
+  if (!S_ctx || !aligned(S_ctx, 16)) return OLA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return from_cuda(cudaGetLastError());
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return OLA_ERR_CUDA;
+  if (prop.major != 10) return OLA_ERR_UNSUPPORTED;
+  if (geom->path == OLA_PATH_REPLAY) {
+    size_t smem = geom->math == OLA_MATH_TENSOR
+                      ? replay_tc_smem(geom->d_k, geom->d_v, geom->B, geom->T_max)
+                      : replay_simt_smem(geom->d_k, geom->d_v, geom->T_max);
+    if (smem > size_t(prop.sharedMemPerBlockOptin)) return OLA_ERR_UNSUPPORTED;
+  }
+
+  ola_ctx* h = new (std::nothrow) ola_ctx();
+  if (!h) return OLA_ERR_OOM;
+  h->g = *geom;
+  h->device = dev;
+  h->t = 0;
+  h->sticky = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  const Sizes z = sizes_of(geom);
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess) e = dev_alloc(&h->S, z.S);
+  if (e == cudaSuccess) e = dev_alloc(&h->S_hi, z.S_split);
+  if (e == cudaSuccess) e = dev_alloc(&h->S_lo, z.S_split);
+  if (e == cudaSuccess) e = dev_alloc(&h->W, z.W);
+  if (e == cudaSuccess) e = dev_alloc(&h->Kr, z.Kr);
+  if (e == cudaSuccess) e = dev_alloc(&h->A, z.A);
+  if (e == cudaSuccess) e = dev_alloc(&h->C, z.C);
+  if (e == cudaSuccess) e = dev_alloc(&h->FS[0], z.FS);
+  if (e == cudaSuccess) e = dev_alloc(&h->FS[1], z.FS);
+  if (e == cudaSuccess) e = dev_alloc(&h->err, z.err);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h->S, S_ctx, z.S, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, z.err, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->C, 0, z.C, st);
+  if (e == cudaSuccess && geom->math == OLA_MATH_TENSOR) {
+    const int RH = geom->R * geom->H;
+    e = launch_split_state(h->S, h->S_hi, h->S_lo, RH, geom->d_k, geom->d_v, st);
+    if (e == cudaSuccess && (!make_state_map(&h->m_hi, h->S_hi, RH, geom->d_k, geom->d_v) ||
+                             !make_state_map(&h->m_lo, h->S_lo, RH, geom->d_k, geom->d_v)))
+      e = cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) {
+    ola_status rs = from_cuda(e);
+    cudaStreamSynchronize(st);
+    free_all(h);
+    delete h;
+    return rs;
+  }
+  *out = h;
+  return OLA_OK;
+}
+
+ola_status ola_step(ola_handle h, const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, const int32_t* parent_idx, float* out_o, void* stream) {
+  if (!h) return OLA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !g || !beta || !parent_idx || !out_o) return OLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out_o, 16) ||
+      !aligned(g, 4) || !aligned(beta, 4) || !aligned(parent_idx, 4))
+    return OLA_ERR_INVALID_ARG;
+  if (h->sticky) return static_cast<ola_status>(h->sticky);
+  if (h->t >= h->g.T_max) return OLA_ERR_CAPACITY;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  StepArgs a = make_args(h, q, k, v, g, beta, parent_idx, out_o);
+  cudaError_t e;
+  if (h->g.path == OLA_PATH_FULLSTATE)
+    e = launch_fullstate(a, h->g.in_dtype, st);
+  else if (h->g.math == OLA_MATH_TENSOR)
+    e = launch_replay_tc(a, h->m_hi, h->m_lo, st);
+  else
+    e = launch_replay_simt(a, h->g.in_dtype, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  h->t += 1;
+  h->last_stream = st;
+  return OLA_OK;
+}
+
+ola_status ola_step_host(ola_handle h, const void* q, const void* k, const void* v,
+                         const float* g, const float* beta, const int32_t* parent_idx,
+                         float* out_o, void* stream) {
+  if (!h) return OLA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !g || !beta || !parent_idx || !out_o) return OLA_ERR_INVALID_ARG;
+  const size_t R = h->g.R, B = h->g.B, H = h->g.H;
+  const size_t e = h->g.in_dtype == OLA_BF16 ? 2 : 4;
+  const size_t bytes[7] = {R * B * H * h->g.d_k * e, R * B * H * h->g.d_k * e,
+                           R * B * H * h->g.d_v * e, R * B * H * 4, R * B * H * 4, R * B * 4,
+                           R * B * H * h->g.d_v * 4};
+  for (int i = 0; i < 7; ++i)
+    if (!h->st[i]) {
+      cudaError_t ce = cudaMalloc(&h->st[i], bytes[i]);
+      if (ce != cudaSuccess) return from_cuda(ce);
+    }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const void* src[6] = {q, k, v, g, beta, parent_idx};
+  for (int i = 0; i < 6; ++i) {
+    cudaError_t ce = cudaMemcpyAsync(h->st[i], src[i], bytes[i], cudaMemcpyHostToDevice, st);
+    if (ce != cudaSuccess) return from_cuda(ce);
+  }
+  ola_status s = ola_step(h, h->st[0], h->st[1], h->st[2], static_cast<const float*>(h->st[3]),
+                          static_cast<const float*>(h->st[4]),
+                          static_cast<const int32_t*>(h->st[5]), static_cast<float*>(h->st[6]),
+                          stream);
+  if (s != OLA_OK) return s;
+  cudaError_t ce = cudaMemcpyAsync(out_o, h->st[6], bytes[6], cudaMemcpyDeviceToHost, st);
+  if (ce != cudaSuccess) return from_cuda(ce);
+  return from_cuda(cudaStreamSynchronize(st));
+}
+
+ola_status ola_reset(ola_handle h) {
+  if (!h) return OLA_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemsetAsync(h->err, 0, 16, h->last_stream);
+  if (e != cudaSuccess) return from_cuda(e);
+  h->t = 0;
+  h->sticky = 0;
+  return OLA_OK;
+}
+
+int32_t ola_current_step(ola_handle h) { return h ? h->t : -1; }
+
+ola_status ola_get_ancestry(ola_handle h, int32_t* out, void* stream) {
+  if (!h || !out || h->t == 0) return OLA_ERR_INVALID_ARG;
+  const size_t t = h->t, Tm = h->g.T_max;
+  const int32_t* src = h->C + size_t(t - 1) * h->g.R * h->g.B * Tm;
+  cudaError_t e = cudaMemcpy2DAsync(out, t * 4, src, Tm * 4, t * 4, size_t(h->g.R) * h->g.B,
+                                    cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream));
+  return from_cuda(e);
+}
+
+ola_status ola_get_error(ola_handle h) {
+  if (!h) return OLA_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(h->last_stream);
+  if (e != cudaSuccess) return from_cuda(e);
+  int w[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(w, h->err, 16, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (w[0] != 0) h->sticky = w[0];
+  return static_cast<ola_status>(h->sticky);
+}
+
+ola_status ola_destroy(ola_handle h) {
+  if (!h) return OLA_OK;
+  cudaStreamSynchronize(h->last_stream);
+  free_all(h);
+  delete h;
+  return OLA_OK;
+}
+
+ola_status ola_prefill(int32_t R, int32_t H, int32_t d_k, int32_t d_v, int32_t P,
+                       int32_t in_dtype, const void* k, const void* v, const float* g,
+                       const float* beta, float* S_out, void* stream) {
+  if (R < 1 || H < 1 || P < 0) return OLA_ERR_INVALID_ARG;
+  if (in_dtype != OLA_F32 && in_dtype != OLA_BF16) return OLA_ERR_INVALID_ARG;
+  if (!pow2_width(d_k) || !pow2_width(d_v)) return OLA_ERR_UNSUPPORTED;
+  if (!S_out || !aligned(S_out, 16)) return OLA_ERR_INVALID_ARG;
+  if (P > 0 && (!k || !v || !g || !beta)) return OLA_ERR_INVALID_ARG;
+  return from_cuda(launch_prefill(R, H, d_k, d_v, P, in_dtype, k, v, g, beta, S_out,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

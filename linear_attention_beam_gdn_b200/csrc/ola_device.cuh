@@ -1,0 +1,256 @@
+// Device-side definitions shared by the library's kernels: the argument block of one decode
+// step, record/ancestry indexing, input loads, warp reductions, bounded waits, and thin
+// inline-PTX wrappers for mbarrier, TMA and tcgen05 (sm_100a).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ola.h"
+
+namespace ola {
+
+// Everything one decode step needs. Record storage (the transition records of every beam,
+// appended once and never moved):
+//   W  [T_max][R][H][B][d_v] fp32   w_t = beta (v - alpha u)
+//   Kr [T_max][R][H][B][d_k] in_dtype  copy of k_t
+//   A  [T_max][R][H][B]      fp32   alpha_t = exp(g_t)
+//   C  [T_max][R][B][T_max]  int32  chain rows: C[t-1][r][b][s] = beam index of the record at
+//                                   step s+1 on beam b's chain after step t (s < t)
+// Slot t-1 holds step t.
+struct StepArgs {
+  int R, H, d_k, d_v, B, T_max;
+  int t;                        // step being computed, 1-based
+  const void* q;                // [R][B][H][d_k]
+  const void* k;                // [R][B][H][d_k]
+  const void* v;                // [R][B][H][d_v]
+  const float* g;               // [R][B][H]
+  const float* beta;            // [R][B][H]
+  const int* parent;            // [R][B]
+  float* o;                     // [R][B][H][d_v]
+  const float* S;               // [R][H][d_v][d_k] shared state (fp32)
+  float* W;
+  void* Kr;
+  float* A;
+  int* C;
+  const float* FS_prev;         // FullState: [R][H][B][d_v][d_k] states of step t-1
+  float* FS_cur;                // FullState: states of step t
+  int* err;                     // device error word: [0] code, [1] detail, [2] step
+};
+
+__host__ __device__ __forceinline__ size_t rec_index(const StepArgs& a, int slot, int r, int h,
+                                                     int b) {
+  return ((size_t(slot) * a.R + r) * a.H + h) * size_t(a.B) + b;
+}
+__host__ __device__ __forceinline__ size_t chain_row(const StepArgs& a, int slot, int r, int b) {
+  return ((size_t(slot) * a.R + r) * size_t(a.B) + b) * size_t(a.T_max);
+}
+
+// First error wins; later ones are dropped. Never traps.
+__device__ __forceinline__ void report_error(int* err, int code, int detail, int step) {
+  if (atomicCAS(err, 0, code) == 0) {
+    err[1] = detail;
+    err[2] = step;
+  }
+}
+
+// Parent of new beam b of request r at step t, validated and clamped.
+__device__ __forceinline__ int checked_parent(const StepArgs& a, int r, int b) {
+  int p = a.parent[size_t(r) * a.B + b];
+  bool bad = (a.t == 1) ? (p != 0) : (p < 0 || p >= a.B);
+  if (bad) {
+    report_error(a.err, OLA_ERR_BAD_PARENT, p, a.t);
+    p = 0;
+  }
+  return p;
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ float ld_in(const void* base, size_t idx) {
+  return to_f32(static_cast<const T*>(base)[idx]);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+// Sum over aligned groups of `width` lanes (width a power of two <= 32).
+__device__ __forceinline__ float group_sum(float x, int width) {
+  for (int off = width >> 1; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Every spin-wait in this library gives up after this long and reports OLA_ERR_TIMEOUT.
+constexpr uint64_t kWaitLimitNs = 1500ull * 1000ull * 1000ull;   // 1.5 s
+
+// ------------------------------------------------------------------ mbarrier (shared::cta)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity to complete. Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 0; it < (1u << 30); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u && global_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return false;
+}
+
+// ------------------------------------------------------------------ TMA (no multicast)
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+      "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------------------------ tcgen05 (cta_group::1)
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* holder_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(holder_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16 operands, fp32 accumulate).
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive (once) on an mbarrier when every tcgen05 operation issued so far by this thread
+// has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major operand stored with the 128-byte swizzle as TMA
+// writes it: rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), leading
+// byte offset unused for this layout (encoded 1), descriptor version 1 (bits 46-47), layout
+// type 2 = 128B swizzle (bits 61-63).
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= uint64_t((smem_addr & 0x3FFFFu) >> 4);      // start address
+  d |= uint64_t(1) << 16;                           // leading byte offset (16 B)
+  d |= uint64_t(1024 >> 4) << 32;                   // stride byte offset
+  d |= uint64_t(1) << 46;                           // version
+  d |= uint64_t(2) << 61;                           // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4)                                  // D format: f32
+         | (1u << 7)                                // A format: bf16
+         | (1u << 10)                               // B format: bf16
+         | (uint32_t(N >> 3) << 17)                 // N / 8
+         | (uint32_t(M >> 4) << 24);                // M / 16
+}
+
+// Two loads of 32 lanes x 8 consecutive 32-bit columns from tensor memory (one lane per
+// thread) followed by the wait, in one asm statement so that no instruction can read the
+// destination registers before the asynchronous loads have landed.
+__device__ __forceinline__ void tmem_ld8x2(uint32_t ta, uint32_t tb, float (&xa)[8],
+                                           float (&xb)[8]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%16];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8, %9, %10, %11, %12, %13, %14, %15}, [%17];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(ta), "r"(tb)
+      : "memory");
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    xa[j] = __uint_as_float(r[j]);
+    xb[j] = __uint_as_float(r[8 + j]);
+  }
+}
+
+}  // namespace ola

@@ -1,0 +1,232 @@
+"""Parity of the CUDA library (through its C ABI) with the FP64 oracle on seeded inputs.
+
+Tolerances (max-abs over every step, request, beam, head and component of o):
+1e-4 on the fp32 paths, 2e-3 on the bf16-operand tensor-core path; ancestry bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_beam_gdn_b200 as ola
+import oracle
+import workloads as wl
+from helpers import (PATHS, max_abs, oracle_outputs, oracle_prefill_all, run_library,
+                     small_problem, stack_f64, tol_for)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_ok):
+    from linear_attention_beam_gdn_b200 import build
+    build.build()
+    torch.cuda.init()
+
+
+def _check(w, paths, S32, steps, dev_steps, parents, ref=None):
+    ref = oracle_outputs(S32, steps, parents) if ref is None else ref
+    anc_ref = oracle.ancestry_table(parents)
+    for path in paths:
+        o, anc, status = run_library(S32.cuda(), dev_steps, parents, path, w.torch_dtype)
+        assert status == ola.OLA_OK, (path, status)
+        err = max_abs(o, ref)
+        print(f"{w.name} {path}: max-abs {err:.3e}")
+        assert err <= tol_for(path), (path, err)
+        assert np.array_equal(anc, anc_ref), path
+    return ref
+
+
+# ----------------------------------------------------------------------------- prefill
+
+@pytest.mark.parametrize("name", ["tiny", "single_request"])
+def test_prefill_matches_oracle(name):
+    w = wl.WORKLOADS[name]
+    if name == "single_request":
+        w = w.scaled(H=4)
+    prompt = wl.make_prompt(w, "cpu")
+    S_ref = oracle_prefill_all(prompt)
+    dp = {k: v.cuda() for k, v in prompt.items()}
+    S = ola.prefill(dp["k"], dp["v"], dp["g"], dp["beta"])
+    err = max_abs(S.double().cpu().numpy(), S_ref)
+    print(f"prefill {name}: max-abs {err:.3e}")
+    assert err <= 1e-4
+
+
+def test_prefill_zero_tokens_gives_zero_state():
+    w = wl.WORKLOADS["tiny"].scaled(P=0)
+    k = torch.empty((1, 0, 2, 16), device="cuda")
+    S = ola.prefill(k, torch.empty((1, 0, 2, 16), device="cuda"),
+                    torch.empty((1, 0, 2), device="cuda"), torch.empty((1, 0, 2), device="cuda"))
+    assert torch.count_nonzero(S) == 0
+
+
+# ----------------------------------------------------------------------------- whole workloads
+
+def test_tiny_all_fp32_paths():
+    w = wl.WORKLOADS["tiny"]
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+
+
+def test_single_request_all_paths():
+    w = wl.WORKLOADS["single_request"]
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+
+
+@pytest.mark.parametrize("d_k", [64, 128, 256])
+@pytest.mark.parametrize("d_v", [64, 128, 256])
+def test_geometries_reduced(d_k, d_v):
+    """The nine recurrent geometries at a size the oracle finishes in seconds, with a ragged
+    beam count (not a multiple of any chunk) and several tiles."""
+    w = wl.WORKLOADS[f"sweep_dk{d_k}_dv{d_v}_B64"].scaled(R=2, H=2, B=100, P=128, T=4)
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+
+
+@pytest.mark.parametrize("B", [16, 17, 33, 64, 65, 200])
+def test_ragged_beam_counts(B):
+    w = wl.WORKLOADS["single_request"].scaled(H=2, B=B, P=64, T=3)
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+
+
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_tiny_beam_counts_fp32(B):
+    w = wl.WORKLOADS["tiny"].scaled(B=B, T=4)
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+
+
+def test_max_steps_32():
+    """T_max = 32 (the largest a handle holds): chains as long as a warp."""
+    w = wl.WORKLOADS["single_request"].scaled(H=1, B=24, P=16, T=32)
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+
+
+def test_bf16_inputs_small_widths_fp32_path():
+    w = wl.WORKLOADS["tiny"].scaled(dtype="bf16", d_k=32, d_v=16, B=12)
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+
+
+# ----------------------------------------------------------------------------- properties
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_identical_ancestry_bit_identical(path):
+    """Two beams with the same parent and the same inputs give bit-identical outputs, wherever
+    they sit in the beam array (different chunks / CTAs)."""
+    w = wl.WORKLOADS["single_request"].scaled(H=2, B=130, P=32, T=3)
+    S32, steps, dev_steps, parents = small_problem(w)
+    parents = parents.copy()
+    for t in range(w.T):
+        for key in ("q", "k", "v", "g", "beta"):
+            dev_steps[t][key][:, 129] = dev_steps[t][key][:, 5]
+            dev_steps[t][key][:, 70] = dev_steps[t][key][:, 5]
+        parents[t, :, 129] = parents[t, :, 5]
+        parents[t, :, 70] = parents[t, :, 5]
+    o, _, st = run_library(S32.cuda(), dev_steps, parents, path, w.torch_dtype)
+    assert st == ola.OLA_OK
+    assert np.array_equal(o[:, :, 129], o[:, :, 5])
+    assert np.array_equal(o[:, :, 70], o[:, :, 5])
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_deterministic(path):
+    w = wl.WORKLOADS["single_request"].scaled(H=4, P=32)
+    S32, steps, dev_steps, parents = small_problem(w)
+    o1, a1, _ = run_library(S32.cuda(), dev_steps, parents, path, w.torch_dtype)
+    o2, a2, _ = run_library(S32.cuda(), dev_steps, parents, path, w.torch_dtype)
+    assert np.array_equal(o1, o2) and np.array_equal(a1, a2)
+
+
+def test_replay_agrees_with_fullstate_on_gpu():
+    w = wl.WORKLOADS["single_request"].scaled(H=4, P=256)
+    S32, steps, dev_steps, parents = small_problem(w)
+    o_fs, _, _ = run_library(S32.cuda(), dev_steps, parents, "fullstate", w.torch_dtype)
+    o_rp, _, _ = run_library(S32.cuda(), dev_steps, parents, "replay_fp32", w.torch_dtype)
+    assert max_abs(o_fs, o_rp) <= 1e-4
+
+
+def test_step_host_matches_step():
+    w = wl.WORKLOADS["single_request"].scaled(H=2, P=32, T=3)
+    S32, steps, dev_steps, parents = small_problem(w)
+    o_dev, _, _ = run_library(S32.cuda(), dev_steps, parents, "replay_tensor", w.torch_dtype)
+    dec = ola.Decoder(S32.cuda(), B=w.B, T_max=w.T, in_dtype=w.torch_dtype)
+    try:
+        for t in range(w.T):
+            s = {k: v.pin_memory() for k, v in steps[t].items()}
+            out = torch.empty((w.R, w.B, w.H, w.d_v)).pin_memory()
+            dec.step_host(s["q"], s["k"], s["v"], s["g"], s["beta"],
+                          torch.from_numpy(parents[t]).pin_memory(), out)
+            assert np.array_equal(out.double().numpy(), o_dev[t])
+    finally:
+        dec.close()
+
+
+# ----------------------------------------------------------------------------- errors
+
+def test_bad_parent_is_sticky_and_reset_clears():
+    w = wl.WORKLOADS["single_request"].scaled(H=2, B=32, P=8, T=3)
+    S32, steps, dev_steps, parents = small_problem(w)
+    for path in PATHS:
+        p, m = PATHS[path]
+        dec = ola.Decoder(S32.cuda(), B=w.B, T_max=3, in_dtype=w.torch_dtype, path=p, math=m)
+        try:
+            s = dev_steps[0]
+            bad = torch.zeros((w.R, w.B), dtype=torch.int32, device="cuda")
+            bad[0, 3] = 1                       # step 1 must have parent 0
+            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], bad)
+            assert dec.error() == ola.OLA_ERR_BAD_PARENT
+            with pytest.raises(ola.OlaError) as ei:
+                dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], bad)
+            assert ei.value.status == ola.OLA_ERR_BAD_PARENT
+            dec.reset()
+            assert dec.error() == ola.OLA_OK and dec.t == 0
+            good = torch.zeros((w.R, w.B), dtype=torch.int32, device="cuda")
+            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], good)
+            s1 = dev_steps[1]
+            oob = torch.full((w.R, w.B), w.B, dtype=torch.int32, device="cuda")
+            dec.step(s1["q"], s1["k"], s1["v"], s1["g"], s1["beta"], oob)
+            assert dec.error() == ola.OLA_ERR_BAD_PARENT
+        finally:
+            dec.close()
+
+
+def test_capacity_and_argument_errors():
+    w = wl.WORKLOADS["single_request"].scaled(H=2, B=32, P=8, T=2)
+    S32, steps, dev_steps, parents = small_problem(w)
+    dec = ola.Decoder(S32.cuda(), B=w.B, T_max=2, in_dtype=w.torch_dtype)
+    try:
+        for t in range(2):
+            s = dev_steps[t]
+            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"],
+                     torch.from_numpy(parents[t]).cuda())
+        with pytest.raises(ola.OlaError) as ei:
+            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"],
+                     torch.from_numpy(parents[1]).cuda())
+        assert ei.value.status == ola.OLA_ERR_CAPACITY
+        assert dec.t == 2
+        # misaligned q pointer: rejected on the host, nothing launched
+        out = torch.empty((w.R, w.B, w.H, w.d_v), device="cuda")
+        qbuf = torch.empty(s["q"].numel() + 8, dtype=s["q"].dtype, device="cuda")
+        st = ola.ola_step(dec.handle, qbuf.data_ptr() + 2, s["k"].data_ptr(),
+                          s["v"].data_ptr(), s["g"].data_ptr(), s["beta"].data_ptr(),
+                          torch.from_numpy(parents[1]).cuda().data_ptr(), out.data_ptr(), None)
+        assert st == ola.OLA_ERR_INVALID_ARG
+        assert dec.error() == ola.OLA_OK
+    finally:
+        dec.close()
+
+
+def test_shape_checks_in_binding():
+    w = wl.WORKLOADS["single_request"].scaled(H=2, B=32, P=8, T=2)
+    S32, steps, dev_steps, parents = small_problem(w)
+    with ola.Decoder(S32.cuda(), B=w.B, T_max=2, in_dtype=w.torch_dtype) as dec:
+        s = dev_steps[0]
+        with pytest.raises(ValueError):
+            dec.step(s["q"][:, :16], s["k"], s["v"], s["g"], s["beta"],
+                     torch.zeros((w.R, w.B), dtype=torch.int32, device="cuda"))
+        with pytest.raises(TypeError):
+            dec.step(s["q"].float(), s["k"], s["v"], s["g"], s["beta"],
+                     torch.zeros((w.R, w.B), dtype=torch.int32, device="cuda"))
