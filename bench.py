@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Throughput of beam-parallel Gated DeltaNet decode (projection replay) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload stress]
+    python bench.py --impl reference ...        # the FP64 CPU oracle on the host cores
+
+One bench step = one whole decode of the workload: ola_reset and T ola_step calls over
+every request, beam and head (plan kernel + fused tensor-core replay kernel per call), with
+all inputs resident in HBM. The metric is beam-head decode steps per second, R*H*B*T per
+bench step, summed over ranks (requests are independent: every rank decodes its own batch
+of requests, weak scaling, no collective on the data path; barrier + max over ranks for the
+timing). Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as wl  # noqa: E402
+
+METRIC = "beam-head decode steps/s (GDN projection replay) and % of roofline, 1×B200"
+UNIT = "beam-head-steps/s"
+
+
+# ----------------------------------------------------------------------------- roofline
+
+def algorithmic_bytes_per_step(w: wl.Workload, parents: np.ndarray) -> list:
+    """Compulsory HBM bytes of each decode step t (one ola_step launch), summed over requests
+    and heads: the shared state read once, q/k/v/g/beta read, o written, the new record
+    (w_t fp32, k_t, alpha_t) written, every distinct ancestor record read once, the parent
+    row read and the chain row written."""
+    e = w.elem_bytes
+    dk, dv, B, H = w.d_k, w.d_v, w.B, w.H
+    U = wl.distinct_ancestor_counts(parents)          # [T, R]
+    rec = 4 * dv + e * dk + 4
+    out = []
+    for t in range(w.T):
+        per_rh = 4 * dv * dk + B * ((2 * dk + dv) * e + 8) + 4 * B * dv + B * rec
+        total = w.R * H * per_rh + H * int(U[t].sum()) * rec + w.R * 4 * B * (t + 2)
+        out.append(total)
+    return out
+
+
+def tensor_flops_per_step(w: wl.Workload) -> int:
+    return 4 * w.d_v * w.d_k * w.B * w.R * w.H
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("ola_replay_tc.cu", "ola_plan.cu", "ola_device.cuh"):
+        h.update(open(os.path.join(ROOT, "linear_attention_beam_gdn_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the replay kernel from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "replay_tc_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("kernel_src_sha") != kernel_source_hash() or d.get("workload") != workload:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx,
+                "samples": len(sms), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- oracle baseline
+
+def _oracle_unit_prefill(args):
+    import oracle
+    k, v, g, b = args
+    return oracle.prefill(k, v, g, b)
+
+
+def _oracle_unit_decode(args):
+    import oracle
+    S, q, k, v, g, b, par = args
+    return oracle.full_state_decode(S, q, k, v, g, b, par)
+
+
+def _pool(cores):
+    import multiprocessing as mp
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    os.environ.setdefault("OPENBLAS_NUM_THREADS", "1")
+    os.environ.setdefault("MKL_NUM_THREADS", "1")
+    return mp.get_context("spawn").Pool(cores)
+
+
+def oracle_sample(w: wl.Workload, prompt_units, step_units, parents, pool, cores):
+    """Time the oracle's full-state decode on the sampled (r, h) units (its own fp64 prefill
+    of their prompts runs first, untimed). Returns (seconds, beam-head-steps)."""
+    S = pool.map(_oracle_unit_prefill, prompt_units)
+    jobs = [(S[i],) + tuple(step_units[i]) + (parents[i],) for i in range(len(S))]
+    t0 = time.perf_counter()
+    pool.map(_oracle_unit_decode, jobs)
+    dt = time.perf_counter() - t0
+    return dt, len(jobs) * w.B * w.T
+
+
+def host_units(w, prompt, steps, parents, units):
+    import oracle
+    pu, su, pa = [], [], []
+    for r, h in units:
+        pu.append(tuple(oracle.as_f64(prompt[x][r, :, h]) for x in ("k", "v", "g", "beta")))
+        su.append(tuple(np.stack([oracle.as_f64(s[x][r, :, h]) for s in steps])
+                        for x in ("q", "k", "v", "g", "beta")))
+        pa.append(parents[:, r])
+    return pu, su, pa
+
+
+def sample_units(w, n, seed=7):
+    rng = np.random.default_rng(seed)
+    allu = [(r, h) for r in range(w.R) for h in range(w.H)]
+    idx = rng.permutation(len(allu))[:n]
+    return [allu[i] for i in idx]
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = wl.WORKLOADS[args.workload]
+    cores = len(os.sched_getaffinity(0))
+    n_units = max(2, 2 * cores)
+    pool = _pool(cores)
+    units = sample_units(w, n_units)
+    import torch
+    prompt = wl.make_prompt(w.scaled(R=max(r for r, _ in units) + 1), "cpu")
+    steps = [wl.make_step_inputs(w, t, "cpu", R=max(r for r, _ in units) + 1)
+             for t in range(w.T)]
+    parents = wl.make_parents(w)
+    pu, su, pa = host_units(w, prompt, steps, parents, units)
+    for _ in range(args.warmup):
+        oracle_sample(w, pu[:cores], su[:cores], pa[:cores], pool, cores)
+    times, work = [], 0
+    for _ in range(args.steps):
+        dt, n = oracle_sample(w, pu, su, pa, pool, cores)
+        times.append(dt)
+        work = n
+    pool.close()
+    total = sum(times)
+    value = work * args.steps / total
+    sample = (f"{n_units} of {w.R * w.H} (request, head) units, all {w.B} beams x {w.T} steps; "
+              f"fp64 prefill of those units untimed")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": describe(w), "parallelism": "host cores (process pool)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def describe(w: wl.Workload) -> str:
+    cap = f", <= {w.max_children} children" if w.max_children else ""
+    return (f"{w.name}: R={w.R} requests x H={w.H} heads, d_k={w.d_k}, d_v={w.d_v}, "
+            f"prompt P={w.P}, B={w.B} beams, T={w.T} decode steps, {w.parent_law}"
+            f"({w.zipf_s}) parents{cap}, {w.dtype} q/k/v, fp32 S_ctx")
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import linear_attention_beam_gdn_b200 as ola
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        tt = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        return float(tt.item())
+
+    base = wl.WORKLOADS[args.workload]
+    w = base.scaled(seed=base.seed + 7919 * rank)       # every rank: its own requests
+    cores = len(os.sched_getaffinity(0))
+    pool = None
+    do_cpu = (not args.no_cpu_baseline) and rank == 0 and world == 1
+    if do_cpu:
+        pool = _pool(cores)                              # spawn before the first GPU call
+
+    # ---- inputs resident in HBM; shared state by the library's prefill kernel
+    prompt = wl.make_prompt(w, dev)
+    S = ola.prefill(prompt["k"], prompt["v"], prompt["g"], prompt["beta"])
+    steps = [wl.make_step_inputs(w, t, dev) for t in range(w.T)]
+    parents = wl.make_parents(w)
+    par_dev = [torch.from_numpy(parents[t]).to(dev) for t in range(w.T)]
+    units = sample_units(w, max(2, 2 * cores)) if do_cpu else []
+    host = host_units(w, prompt, steps, parents, units) if do_cpu else None
+    del prompt
+    torch.cuda.synchronize()
+
+    outs = [torch.empty((w.R, w.B, w.H, w.d_v), device=dev) for _ in range(w.T)]
+    stream = torch.cuda.current_stream()
+
+    def decode(dec, evs=None):
+        dec.reset()
+        for t in range(w.T):
+            s = steps[t]
+            if evs is not None:
+                evs[t][0].record(stream)
+            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], par_dev[t], out=outs[t])
+            if evs is not None:
+                evs[t][1].record(stream)
+
+    dec = ola.Decoder(S, B=w.B, T_max=w.T, in_dtype=w.torch_dtype, path=ola.OLA_PATH_REPLAY,
+                      math=ola.OLA_MATH_TENSOR)
+    for _ in range(args.warmup):
+        decode(dec)
+    torch.cuda.synchronize()
+    st = dec.error()
+    if st != ola.OLA_OK:
+        raise RuntimeError(f"device error during warm-up: {ola.ola_strerror(st)}")
+
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(w.T)]
+           for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for k in range(K):
+            decode(dec, evs[k])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    clocks = clk.summary()
+    st = dec.error()
+    if st != ola.OLA_OK:
+        raise RuntimeError(f"device error in the timed region: {ola.ola_strerror(st)}")
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    step_ms = np.array([[evs[k][t][0].elapsed_time(evs[k][t][1]) for t in range(w.T)]
+                        for k in range(K)])
+    per_launch_ms = step_ms.mean(axis=0)               # ola_step t, averaged over K
+    units_per_step = w.R * w.H * w.B * w.T
+    value = world * units_per_step * K / (ms / 1e3)
+
+    # ---- roofline of the step kernel
+    peaks = measured_peaks()
+    bytes_t = algorithmic_bytes_per_step(w, parents)
+    achieved = sum(bytes_t) / (per_launch_ms.sum() / 1e3) / 1e9
+    flops = tensor_flops_per_step(w) * w.T
+    tensor_time = flops / (peaks["bf16_tflops"] * 1e12)
+    hbm_time = sum(bytes_t) / (peaks["hbm_gbs"] * 1e9)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"],
+                "traffic": recorded_traffic(w.name),
+                "kernel": "ola_step (ola::plan_kernel + ola::replay_tc_kernel<128,128>)",
+                "algorithmic_bytes_per_decode": int(sum(bytes_t)),
+                "algorithmic_bytes_per_launch": [int(b) for b in bytes_t],
+                "launch_ms": [round(float(x), 4) for x in per_launch_ms],
+                "t_roof_ms": 1e3 * max(tensor_time, hbm_time),
+                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"}
+
+    result = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+              "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+              "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+              "data": "synthetic",
+              "config": {"workload": describe(w), "R": w.R, "H": w.H, "d_k": w.d_k,
+                         "d_v": w.d_v, "B": w.B, "T": w.T, "P": w.P,
+                         "path": "replay, tcgen05 tensor cores (bf16 hi/lo S_ctx, fp32 "
+                                 "accumulate and epilogue)",
+                         "l2": "no flush: each decode step streams ~1.4 GB (> 126 MB L2)",
+                         "parallelism": f"replicas x{world} (requests sharded, no collective)"},
+              "roofline": roofline, "clocks": clocks,
+              "gpu_launches": 2 * w.T * K}
+
+    # ---- in-library comparisons on the same inputs (not part of the metric)
+    comps = {}
+    if not args.no_compare:
+        for name, p, m, reps in (("replay_fp32", ola.OLA_PATH_REPLAY, ola.OLA_MATH_FP32, 2),
+                                 ("fullstate", ola.OLA_PATH_FULLSTATE, ola.OLA_MATH_FP32, 2)):
+            try:
+                d2 = ola.Decoder(S, B=w.B, T_max=w.T, in_dtype=w.torch_dtype, path=p, math=m)
+            except ola.OlaError as ex:
+                comps[name] = {"skipped": str(ex)}
+                continue
+            decode(d2)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                decode(d2)
+            b.record(stream)
+            torch.cuda.synchronize()
+            mms = max_over_ranks(a.elapsed_time(b)) / reps
+            comps[name] = {"ms_per_step": mms, "value": world * units_per_step / (mms / 1e3),
+                           "replay_tensor_speedup": mms / (ms / K)}
+            d2.close()
+            del d2
+            torch.cuda.empty_cache()
+    result["compare"] = comps
+
+    # ---- end to end through the host-buffer entry point (pinned memory)
+    if not args.no_e2e:
+        hs = [{k: v.cpu().pin_memory() for k, v in s.items()} for s in steps]
+        hp = [torch.from_numpy(parents[t]).pin_memory() for t in range(w.T)]
+        hout = torch.empty((w.R, w.B, w.H, w.d_v), dtype=torch.float32).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for s in hs for v in s.values()) + \
+            sum(p.numel() * 4 for p in hp)
+        d2h = w.T * hout.numel() * 4
+
+        def decode_host():
+            dec.reset()
+            for t in range(w.T):
+                s = hs[t]
+                dec.step_host(s["q"], s["k"], s["v"], s["g"], s["beta"], hp[t], hout)
+
+        decode_host()
+        barrier()
+        t0 = time.perf_counter()
+        for _ in range(args.e2e_steps):
+            decode_host()
+        dt = max_over_ranks(time.perf_counter() - t0)
+        result["e2e"] = {"value": world * units_per_step * args.e2e_steps / dt, "unit": UNIT,
+                         "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                         "ms_per_step": 1e3 * dt / args.e2e_steps,
+                         "via": "ola_step_host (host buffers, one cudaMemcpyAsync per tensor)"}
+        if dec.error() != ola.OLA_OK:
+            raise RuntimeError("device error in the end-to-end run")
+        del hs, hp, hout
+
+    dec.close()
+
+    # ---- CPU oracle baseline (rank 0, N = 1)
+    if do_cpu:
+        pu, su, pa = host
+        dt, n = oracle_sample(w, pu, su, pa, pool, cores)
+        pool.close()
+        result["cpu_baseline"] = {
+            "value": n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(pu)} of {w.R * w.H} (request, head) units of this workload, all "
+                      f"{w.B} beams x {w.T} steps, fp64 full-state recurrence; the units' "
+                      f"fp64 prefill untimed", "seconds": dt}
+
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="stress", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-compare", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warm-up raised to 3", file=sys.stderr)
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

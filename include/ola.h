@@ -76,7 +76,7 @@ typedef struct {
   int32_t H;          /* heads, >= 1 */
   int32_t d_k;        /* key width: 16, 32, 64, 128 or 256 (TENSOR: 64, 128, 256) */
   int32_t d_v;        /* value width: 16, 32, 64, 128 or 256 (TENSOR: 64, 128, 256) */
-  int32_t B;          /* beams per request, 1..4096 (TENSOR: >= 16) */
+  int32_t B;          /* beams per request, 1..4096 (TENSOR: T_max*R*H*B < 2^31) */
   int32_t T_max;      /* decode steps the handle can hold, 1..32 */
   int32_t in_dtype;   /* OLA_F32 or OLA_BF16 (TENSOR: OLA_BF16) */
   int32_t path;       /* OLA_PATH_REPLAY or OLA_PATH_FULLSTATE */

@@ -37,6 +37,9 @@ struct ola_ctx {
   float* A = nullptr;
   int* C = nullptr;
   float* FS[2] = {nullptr, nullptr};
+  int* perm = nullptr;       // [2][R][B] depth-first order of the current step and the
+                             // parent of the beam at each position (tensor path)
+  int* rank = nullptr;       // [2][R][B] depth-first position of each beam, by step parity
   int* err = nullptr;
   CUtensorMap m_hi, m_lo;
   // staging buffers of ola_step_host (allocated on first use)
@@ -61,14 +64,16 @@ ola_status validate(const ola_geometry* g) {
   if (int64_t(g->R) * g->H * g->B > (int64_t(1) << 30)) return OLA_ERR_UNSUPPORTED;
   if (g->math == OLA_MATH_TENSOR) {
     if (g->path != OLA_PATH_REPLAY || g->in_dtype != OLA_BF16) return OLA_ERR_UNSUPPORTED;
-    if (!tc_width(g->d_k) || !tc_width(g->d_v) || g->B < 16) return OLA_ERR_UNSUPPORTED;
+    if (!tc_width(g->d_k) || !tc_width(g->d_v)) return OLA_ERR_UNSUPPORTED;
+    // record rows are 32-bit indices in the tensor-core kernel
+    if (int64_t(g->T_max) * g->R * g->H * g->B >= (int64_t(1) << 31)) return OLA_ERR_UNSUPPORTED;
   }
   return OLA_OK;
 }
 
 struct Sizes {
-  size_t S, S_split, W, Kr, A, C, FS, err;
-  size_t total() const { return S + 2 * S_split + W + Kr + A + C + 2 * FS + err; }
+  size_t S, S_split, W, Kr, A, C, FS, perm, rank, err;
+  size_t total() const { return S + 2 * S_split + W + Kr + A + C + 2 * FS + perm + rank + err; }
 };
 
 Sizes sizes_of(const ola_geometry* g) {
@@ -83,6 +88,8 @@ Sizes sizes_of(const ola_geometry* g) {
   z.A = rep ? T * R * H * B * 4 : 0;
   z.C = T * R * B * T * 4;
   z.FS = rep ? 0 : R * H * B * dv * dk * 4;
+  z.perm = g->math == OLA_MATH_TENSOR ? 2 * R * B * 4 : 0;
+  z.rank = g->math == OLA_MATH_TENSOR ? 2 * R * B * 4 : 0;
   z.err = 16;
   return z;
 }
@@ -104,7 +111,8 @@ cudaError_t dev_alloc(T** p, size_t bytes) {
 }
 
 void free_all(ola_ctx* h) {
-  void* ptrs[] = {h->S, h->S_hi, h->S_lo, h->W, h->Kr, h->A, h->C, h->FS[0], h->FS[1], h->err};
+  void* ptrs[] = {h->S,     h->S_hi,  h->S_lo, h->W,    h->Kr,  h->A,
+                  h->C,     h->FS[0], h->FS[1], h->perm, h->rank, h->err};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (void* p : h->st)
@@ -135,6 +143,11 @@ StepArgs make_args(ola_ctx* h, const void* q, const void* k, const void* v, cons
   a.C = h->C;
   a.FS_prev = h->FS[(a.t + 1) & 1];   // states of step t-1 (unused at t = 1)
   a.FS_cur = h->FS[a.t & 1];
+  const size_t RB = size_t(h->g.R) * h->g.B;
+  a.perm = h->perm;
+  a.pparent = h->perm ? h->perm + RB : nullptr;
+  a.rank_prev = h->rank ? h->rank + ((a.t + 1) & 1) * RB : nullptr;
+  a.rank_cur = h->rank ? h->rank + (a.t & 1) * RB : nullptr;
   a.err = h->err;
   return a;
 }
@@ -205,6 +218,8 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
   if (e == cudaSuccess) e = dev_alloc(&h->C, z.C);
   if (e == cudaSuccess) e = dev_alloc(&h->FS[0], z.FS);
   if (e == cudaSuccess) e = dev_alloc(&h->FS[1], z.FS);
+  if (e == cudaSuccess) e = dev_alloc(&h->perm, z.perm);
+  if (e == cudaSuccess) e = dev_alloc(&h->rank, z.rank);
   if (e == cudaSuccess) e = dev_alloc(&h->err, z.err);
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->S, S_ctx, z.S, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, z.err, st);

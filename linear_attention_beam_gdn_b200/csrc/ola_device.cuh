@@ -37,6 +37,10 @@ struct StepArgs {
   int* C;
   const float* FS_prev;         // FullState: [R][H][B][d_v][d_k] states of step t-1
   float* FS_cur;                // FullState: states of step t
+  int* perm;                    // [R][B] beam at each depth-first position of step t
+  int* pparent;                 // [R][B] parent (clamped) of the beam at each position
+  const int* rank_prev;         // [R][B] depth-first position of each beam of step t-1
+  int* rank_cur;                // [R][B] depth-first position of each beam of step t
   int* err;                     // device error word: [0] code, [1] detail, [2] step
 };
 
@@ -109,6 +113,16 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy
+// (tcgen05.mma operand reads, TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 

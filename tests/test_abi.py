@@ -46,8 +46,8 @@ def _geom(**kw):
     (dict(B=5000), ola.OLA_ERR_UNSUPPORTED),
     (dict(math=ola.OLA_MATH_TENSOR), ola.OLA_ERR_UNSUPPORTED),                 # fp32 inputs
     (dict(math=ola.OLA_MATH_TENSOR, in_dtype=ola.OLA_BF16), ola.OLA_ERR_UNSUPPORTED),  # d=16
-    (dict(math=ola.OLA_MATH_TENSOR, in_dtype=ola.OLA_BF16, d_k=128, d_v=128, B=8),
-     ola.OLA_ERR_UNSUPPORTED),                                                  # B < 16
+    (dict(math=ola.OLA_MATH_TENSOR, in_dtype=ola.OLA_BF16, d_k=128, d_v=128, B=4096, R=8192,
+          H=2, T_max=32), ola.OLA_ERR_UNSUPPORTED),                             # 32-bit rows
     (dict(math=ola.OLA_MATH_TENSOR, in_dtype=ola.OLA_BF16, d_k=128, d_v=128, B=16,
           path=ola.OLA_PATH_FULLSTATE), ola.OLA_ERR_UNSUPPORTED),
 ])
@@ -68,6 +68,10 @@ def test_workspace_bytes_formula(L):
     gf = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, path=ola.OLA_PATH_FULLSTATE)
     expect_fs = R * H * dv * dk * 4 + 2 * R * H * B * dv * dk * 4 + T * R * B * T * 4 + 16
     assert ola.ola_workspace_bytes(gf) == expect_fs
+    gt = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, in_dtype=ola.OLA_BF16,
+               math=ola.OLA_MATH_TENSOR)
+    split = 2 * R * H * 128 * dk * 2
+    assert ola.ola_workspace_bytes(gt) == expect + split + 2 * R * B * 4 + 2 * R * B * 4
 
 
 def test_null_arguments(L):

@@ -90,6 +90,13 @@ def test_ragged_beam_counts(B):
     _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
 
 
+@pytest.mark.parametrize("B", [1, 5, 31, 32, 63])
+def test_small_beam_counts_all_paths(B):
+    w = wl.WORKLOADS["single_request"].scaled(H=2, B=B, P=32, T=4)
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+
+
 @pytest.mark.parametrize("B", [1, 3, 8])
 def test_tiny_beam_counts_fp32(B):
     w = wl.WORKLOADS["tiny"].scaled(B=B, T=4)
