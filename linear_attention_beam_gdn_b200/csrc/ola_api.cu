@@ -17,6 +17,10 @@ size_t replay_simt_smem(int d_k, int d_v, int T_max);
 cudaError_t launch_replay_tc(const StepArgs& a, const CUtensorMap& mhi, const CUtensorMap& mlo,
                              cudaStream_t stream);
 size_t replay_tc_smem(int d_k, int d_v, int B, int T_max);
+cudaError_t launch_replay_pos(const StepArgs& a, const CUtensorMap& mhi, const CUtensorMap& mlo,
+                              cudaStream_t stream);
+size_t replay_pos_smem(int d_k, int d_v, int T_max);
+bool replay_pos_supported(int d_k, int d_v);
 bool make_state_map(CUtensorMap* map, const void* base, int RH, int d_k, int d_v);
 cudaError_t launch_split_state(const float* S, void* hi, void* lo, int RH, int d_k, int d_v,
                                cudaStream_t stream);
@@ -40,6 +44,7 @@ struct ola_ctx {
   int* perm = nullptr;       // [2][R][B] depth-first order of the current step and the
                              // parent of the beam at each position (tensor path)
   int* rank = nullptr;       // [2][R][B] depth-first position of each beam, by step parity
+  int* pchain = nullptr;     // [R][B][T_max] parent chain by depth-first position
   int* err = nullptr;
   CUtensorMap m_hi, m_lo;
   // staging buffers of ola_step_host (allocated on first use)
@@ -72,8 +77,10 @@ ola_status validate(const ola_geometry* g) {
 }
 
 struct Sizes {
-  size_t S, S_split, W, Kr, A, C, FS, perm, rank, err;
-  size_t total() const { return S + 2 * S_split + W + Kr + A + C + 2 * FS + perm + rank + err; }
+  size_t S, S_split, W, Kr, A, C, FS, perm, rank, pchain, err;
+  size_t total() const {
+    return S + 2 * S_split + W + Kr + A + C + 2 * FS + perm + rank + pchain + err;
+  }
 };
 
 Sizes sizes_of(const ola_geometry* g) {
@@ -90,6 +97,7 @@ Sizes sizes_of(const ola_geometry* g) {
   z.FS = rep ? 0 : R * H * B * dv * dk * 4;
   z.perm = g->math == OLA_MATH_TENSOR ? 2 * R * B * 4 : 0;
   z.rank = g->math == OLA_MATH_TENSOR ? 2 * R * B * 4 : 0;
+  z.pchain = g->math == OLA_MATH_TENSOR ? R * B * T * 4 : 0;
   z.err = 16;
   return z;
 }
@@ -112,7 +120,7 @@ cudaError_t dev_alloc(T** p, size_t bytes) {
 
 void free_all(ola_ctx* h) {
   void* ptrs[] = {h->S,     h->S_hi,  h->S_lo, h->W,    h->Kr,  h->A,
-                  h->C,     h->FS[0], h->FS[1], h->perm, h->rank, h->err};
+                  h->C,     h->FS[0], h->FS[1], h->perm, h->rank, h->pchain, h->err};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (void* p : h->st)
@@ -146,6 +154,7 @@ StepArgs make_args(ola_ctx* h, const void* q, const void* k, const void* v, cons
   const size_t RB = size_t(h->g.R) * h->g.B;
   a.perm = h->perm;
   a.pparent = h->perm ? h->perm + RB : nullptr;
+  a.pchain = h->pchain;
   a.rank_prev = h->rank ? h->rank + ((a.t + 1) & 1) * RB : nullptr;
   a.rank_cur = h->rank ? h->rank + (a.t & 1) * RB : nullptr;
   a.err = h->err;
@@ -193,9 +202,11 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
   if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return OLA_ERR_CUDA;
   if (prop.major != 10) return OLA_ERR_UNSUPPORTED;
   if (geom->path == OLA_PATH_REPLAY) {
-    size_t smem = geom->math == OLA_MATH_TENSOR
-                      ? replay_tc_smem(geom->d_k, geom->d_v, geom->B, geom->T_max)
-                      : replay_simt_smem(geom->d_k, geom->d_v, geom->T_max);
+    size_t smem = geom->math != OLA_MATH_TENSOR
+                      ? replay_simt_smem(geom->d_k, geom->d_v, geom->T_max)
+                  : replay_pos_supported(geom->d_k, geom->d_v)
+                      ? replay_pos_smem(geom->d_k, geom->d_v, geom->T_max)
+                      : replay_tc_smem(geom->d_k, geom->d_v, geom->B, geom->T_max);
     if (smem > size_t(prop.sharedMemPerBlockOptin)) return OLA_ERR_UNSUPPORTED;
   }
 
@@ -220,6 +231,7 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
   if (e == cudaSuccess) e = dev_alloc(&h->FS[1], z.FS);
   if (e == cudaSuccess) e = dev_alloc(&h->perm, z.perm);
   if (e == cudaSuccess) e = dev_alloc(&h->rank, z.rank);
+  if (e == cudaSuccess) e = dev_alloc(&h->pchain, z.pchain);
   if (e == cudaSuccess) e = dev_alloc(&h->err, z.err);
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->S, S_ctx, z.S, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, z.err, st);
@@ -256,6 +268,8 @@ ola_status ola_step(ola_handle h, const void* q, const void* k, const void* v, c
   cudaError_t e;
   if (h->g.path == OLA_PATH_FULLSTATE)
     e = launch_fullstate(a, h->g.in_dtype, st);
+  else if (h->g.math == OLA_MATH_TENSOR && replay_pos_supported(h->g.d_k, h->g.d_v))
+    e = launch_replay_pos(a, h->m_hi, h->m_lo, st);
   else if (h->g.math == OLA_MATH_TENSOR)
     e = launch_replay_tc(a, h->m_hi, h->m_lo, st);
   else

@@ -39,6 +39,7 @@ struct StepArgs {
   float* FS_cur;                // FullState: states of step t
   int* perm;                    // [R][B] beam at each depth-first position of step t
   int* pparent;                 // [R][B] parent (clamped) of the beam at each position
+  int* pchain;                  // [R][B][T_max] the parent's chain, by depth-first position
   const int* rank_prev;         // [R][B] depth-first position of each beam of step t-1
   int* rank_cur;                // [R][B] depth-first position of each beam of step t
   int* err;                     // device error word: [0] code, [1] detail, [2] step
@@ -173,6 +174,17 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
       "r"(c3)
+      : "memory");
+}
+
+// Plain bulk copy global -> shared (no tensor map, no multicast): `bytes` a multiple of 16,
+// both addresses 16-byte aligned; completion counted on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -12,7 +12,8 @@
 //     position(b) = #{b' : key(b') < key(b)} + #{b' < b : key(b') = key(b)}.
 // Children of one parent become contiguous and parents keep their own depth-first order, so
 // by induction the order is a depth-first order of the whole tree. Outputs: perm[r][pos] = b,
-// pparent[r][pos] = parent of that beam, and rank_cur[r][b] = pos (the next step's keys).
+// pparent[r][pos] = parent of that beam, pchain[r][pos][:] = that parent's chain of record
+// beam indices, and rank_cur[r][b] = pos (the next step's keys).
 // Out-of-range parents are clamped to 0 and reported (OLA_ERR_BAD_PARENT), exactly as the
 // decode kernels do.
 #include <limits.h>
@@ -52,6 +53,11 @@ __global__ void __launch_bounds__(512) plan_kernel(StepArgs a) {
     a.perm[size_t(r) * B + pos] = b;
     a.pparent[size_t(r) * B + pos] = pbuf[b];
     a.rank_cur[size_t(r) * B + b] = pos;
+    // the parent's chain, stored by position so a decode CTA reads it without first
+    // resolving the beam and its parent
+    if (a.pchain != nullptr)
+      for (int s = 0; s < a.t - 1; ++s)
+        a.pchain[(size_t(r) * B + pos) * a.T_max + s] = a.C[chain_row(a, a.t - 2, r, pbuf[b]) + s];
   }
 }
 

@@ -71,7 +71,8 @@ def test_workspace_bytes_formula(L):
     gt = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, in_dtype=ola.OLA_BF16,
                math=ola.OLA_MATH_TENSOR)
     split = 2 * R * H * 128 * dk * 2
-    assert ola.ola_workspace_bytes(gt) == expect + split + 2 * R * B * 4 + 2 * R * B * 4
+    assert ola.ola_workspace_bytes(gt) == (expect + split + 2 * R * B * 4 + 2 * R * B * 4 +
+                                           R * B * T * 4)
 
 
 def test_null_arguments(L):
