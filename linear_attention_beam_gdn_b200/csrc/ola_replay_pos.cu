@@ -171,29 +171,58 @@ replay_pos_kernel(const __grid_constant__ CUtensorMap tm_shi,
   const uint32_t tmem = *holder;
 
   // -------------------------------------------------------------------- phase 1
-  int my_b = 0, my_p = 0, my_io = 0;
+  // Round 1: the beams of this warp's positions and their parents' chains (both indexed by
+  // position). Round 2: q_t, k_t rows, g, beta, the chain's alphas. The rows that phases 2 and
+  // 3 will gather (ancestors' k_j and w_j, v) are prefetched into L2 as soon as known.
+  int recs[PPW];
+#pragma unroll
+  for (int jj = 0; jj < PPW; ++jj) {
+    const bool vj = c0 + p0 + jj < a.B;
+    recs[jj] = (vj && lane < n_anc)
+                   ? a.pchain[(size_t(r) * a.B + c0 + p0 + jj) * a.T_max + lane]
+                   : 0;
+  }
+  int my_b = 0, my_io = 0;
   bool my_valid = false;
   if (lane < PPW) {                                // lane j: this warp's position j
     const int pos = c0 + p0 + lane;
     my_valid = pos < a.B;
     if (my_valid) {
       my_b = a.perm[size_t(r) * a.B + pos];
-      my_p = a.pparent[size_t(r) * a.B + pos];
       my_io = (r * a.B + my_b) * a.H + h;
+    }
+  }
+  int rows[PPW];
+  float al[PPW];
+#pragma unroll
+  for (int jj = 0; jj < PPW; ++jj) {
+    const bool vj = c0 + p0 + jj < a.B;
+    rows[jj] = int(rec_index(a, lane < n_anc ? lane : 0, r, h, recs[jj]));
+    al[jj] = (vj && lane < n_anc) ? a.A[rows[jj]] : 1.f;
+    if (vj && lane < n_anc) {
+      const char* kr = reinterpret_cast<const char*>(
+          static_cast<const __nv_bfloat16*>(a.Kr) + size_t(rows[jj]) * DK);
+      const char* wr = reinterpret_cast<const char*>(a.W + size_t(rows[jj]) * DV);
+#pragma unroll
+      for (int c = 0; c < DK * 2; c += 128) prefetch_l2(kr + c);
+#pragma unroll
+      for (int c = 0; c < DV * 4; c += 128) prefetch_l2(wr + c);
     }
   }
   float my_alpha = 0.f, my_beta = 0.f;
   if (lane < PPW && my_valid) {
     my_alpha = expf(a.g[my_io]);
     my_beta = a.beta[my_io];
+    const char* vr = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.v) +
+                                                   size_t(my_io) * DV);
+#pragma unroll
+    for (int c = 0; c < DV * 2; c += 128) prefetch_l2(vr + c);
   }
   KVec qv[PPW], kv[PPW];
-  int recs[PPW];
 #pragma unroll
   for (int jj = 0; jj < PPW; ++jj) {
     const int io = __shfl_sync(0xffffffffu, my_io, jj);
-    const int pj = __shfl_sync(0xffffffffu, my_p, jj);
-    const bool vj = __shfl_sync(0xffffffffu, my_valid ? 1 : 0, jj) != 0;
+    const bool vj = c0 + p0 + jj < a.B;
     const KVec z = {};
     qv[jj] = vj ? reinterpret_cast<const KVec*>(static_cast<const __nv_bfloat16*>(a.q) +
                                                 size_t(io) * DK)[lane]
@@ -201,11 +230,6 @@ replay_pos_kernel(const __grid_constant__ CUtensorMap tm_shi,
     kv[jj] = vj ? reinterpret_cast<const KVec*>(static_cast<const __nv_bfloat16*>(a.k) +
                                                 size_t(io) * DK)[lane]
                 : z;
-    // lane s < n_anc: record (beam index) of ancestor s of position jj (from the plan)
-    recs[jj] = (vj && lane < n_anc)
-                   ? a.pchain[(size_t(r) * a.B + c0 + p0 + jj) * a.T_max + lane]
-                   : 0;
-    (void)pj;
   }
 #pragma unroll
   for (int jj = 0; jj < PPW; ++jj) {
@@ -218,14 +242,6 @@ replay_pos_kernel(const __grid_constant__ CUtensorMap tm_shi,
   }
   // chain table: record rows and alphas (lane s < n_anc); appends; k_t . q_t
   {
-    float al[PPW];
-    int rows[PPW];
-#pragma unroll
-    for (int jj = 0; jj < PPW; ++jj) {
-      const bool vj = __shfl_sync(0xffffffffu, my_valid ? 1 : 0, jj) != 0;
-      rows[jj] = int(rec_index(a, lane < n_anc ? lane : 0, r, h, recs[jj]));
-      al[jj] = (vj && lane < n_anc) ? a.A[rows[jj]] : 1.f;
-    }
 #pragma unroll
     for (int jj = 0; jj < PPW; ++jj) {
       const int pn = p0 + jj;
