@@ -58,7 +58,8 @@ typedef enum {
   OLA_ERR_BAD_PARENT = 4,    /* a parent index was out of range (device-detected, sticky) */
   OLA_ERR_OOM = 5,           /* device allocation failed */
   OLA_ERR_CUDA = 6,          /* a CUDA runtime call failed */
-  OLA_ERR_TIMEOUT = 7        /* a bounded device wait ran out (device-detected, sticky) */
+  OLA_ERR_TIMEOUT = 7,       /* a bounded device wait ran out (device-detected, sticky) */
+  OLA_ERR_SCRATCH_LIMIT = 8  /* ola_decode_noalloc: problem larger than its fixed scratch */
 } ola_status;
 
 /* dtype of q, k, v (and of the prompt's k, v for ola_prefill) */
@@ -161,6 +162,40 @@ ola_status ola_destroy(ola_handle h);
 ola_status ola_prefill(int32_t R, int32_t H, int32_t d_k, int32_t d_v, int32_t P,
                        int32_t in_dtype, const void* k, const void* v, const float* g,
                        const float* beta, float* S_out, void* stream);
+
+/* ------------------------------------------------------------------ allocation-free decode
+ * Not from the pages: the pages have no counterpart of this entry point. It serves callers
+ * that cannot allocate device memory while decoding, e.g. code running inside a CUDA stream
+ * capture (a cudaMalloc there breaks the capture), servers whose device memory is fully
+ * reserved up front by an arena allocator, and latency-critical loops that cannot afford the
+ * implicit synchronisation of an allocation.
+ *
+ * ola_decode_noalloc runs a whole T_max-step decode of one GDN layer on the fp32 CUDA-core
+ * replay path (same results as ola_create + T_max x ola_step + ola_destroy with
+ * path = REPLAY, math = FP32), without creating a handle and without allocating anything:
+ *   geom        : host pointer; path must be OLA_PATH_REPLAY and math OLA_MATH_FP32; T_max is
+ *                 the number of steps decoded; the other limits are those of ola_create.
+ *   S_ctx       : device [R][H][d_v][d_k] fp32 shared state (read only).
+ *   q, k        : device [T_max][R][B][H][d_k] in_dtype;  v : device [T_max][R][B][H][d_v].
+ *   g, beta     : device [T_max][R][B][H] fp32;  parent_idx : device [T_max][R][B] int32.
+ *   out_o       : device [T_max][R][B][H][d_v] fp32 (written).
+ * The transient state (transition records, ancestry rows, error word) lives in one fixed
+ * device array of OLA_NOALLOC_SCRATCH_BYTES inside the library, held by every GPU that loads
+ * the library until the process exits. Problems needing more than that
+ * (ola_noalloc_scratch_bytes) are rejected with OLA_ERR_SCRATCH_LIMIT before anything runs.
+ * Every call shares the array and leaves its contents behind; calls whose work overlaps on
+ * the GPU (different streams, or several host threads) race on it and must be serialised by
+ * the caller. The first call on each device resolves the array's device address (a runtime
+ * query, no allocation); make that first call before any stream capture. The call is
+ * synchronous: it waits for `stream` and returns the device error status (OLA_OK,
+ * OLA_ERR_BAD_PARENT, ...) of this decode. */
+#define OLA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+uint64_t ola_noalloc_scratch_bytes(const ola_geometry* geom);
+
+ola_status ola_decode_noalloc(const ola_geometry* geom, const float* S_ctx, const void* q,
+                              const void* k, const void* v, const float* g, const float* beta,
+                              const int32_t* parent_idx, float* out_o, void* stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

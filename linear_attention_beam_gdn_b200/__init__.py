@@ -25,6 +25,8 @@ HEADER_PATH = os.path.join(os.path.dirname(PKG_DIR), "include", "ola.h")
 
 OLA_OK, OLA_ERR_INVALID_ARG, OLA_ERR_UNSUPPORTED, OLA_ERR_CAPACITY = 0, 1, 2, 3
 OLA_ERR_BAD_PARENT, OLA_ERR_OOM, OLA_ERR_CUDA, OLA_ERR_TIMEOUT = 4, 5, 6, 7
+OLA_ERR_SCRATCH_LIMIT = 8
+OLA_NOALLOC_SCRATCH_BYTES = 16 << 20
 OLA_F32, OLA_BF16 = 0, 1
 OLA_PATH_REPLAY, OLA_PATH_FULLSTATE = 0, 1
 OLA_MATH_FP32, OLA_MATH_TENSOR = 0, 1
@@ -67,6 +69,9 @@ def _declare(L: ctypes.CDLL) -> None:
         "ola_get_error": (i32, [_P]),
         "ola_destroy": (i32, [_P]),
         "ola_prefill": (i32, [i32, i32, i32, i32, i32, i32, _P, _P, _P, _P, _P, _P]),
+        "ola_noalloc_scratch_bytes": (ctypes.c_uint64, [ctypes.POINTER(Geometry)]),
+        "ola_decode_noalloc": (i32, [ctypes.POINTER(Geometry), _P, _P, _P, _P, _P, _P, _P, _P,
+                                     _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -154,6 +159,16 @@ def ola_destroy(h) -> int:
 
 def ola_prefill(R, H, d_k, d_v, P, in_dtype, k, v, g, beta, S_out, stream) -> int:
     return lib().ola_prefill(R, H, d_k, d_v, P, in_dtype, k, v, g, beta, S_out, stream)
+
+
+def ola_noalloc_scratch_bytes(geom: Geometry) -> int:
+    return lib().ola_noalloc_scratch_bytes(ctypes.byref(geom))
+
+
+def ola_decode_noalloc(geom: Geometry, S_ctx, q, k, v, g, beta, parent_idx, out_o,
+                       stream) -> int:
+    return lib().ola_decode_noalloc(ctypes.byref(geom), S_ctx, q, k, v, g, beta, parent_idx,
+                                    out_o, stream)
 
 
 # ------------------------------------------------------------------ torch-facing wrappers

@@ -177,6 +177,7 @@ const char* ola_strerror(ola_status s) {
     case OLA_ERR_OOM: return "device out of memory";
     case OLA_ERR_CUDA: return "CUDA runtime error";
     case OLA_ERR_TIMEOUT: return "bounded device wait timed out";
+    case OLA_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed no-allocation scratch";
   }
   return "unknown status";
 }

@@ -23,7 +23,7 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_version_and_strerror(L):
     assert ola.ola_version() >> 16 == 1
-    for code in range(8):
+    for code in range(9):
         assert ola.ola_strerror(code)
     assert "unknown" in ola.ola_strerror(99)
 
