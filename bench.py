@@ -241,6 +241,24 @@ def describe(w: wl.Workload) -> str:
             f"({w.zipf_s}) parents{cap}, {w.dtype} q/k/v, fp32 S_ctx")
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_workload(base: wl.Workload, rank: int) -> wl.Workload:
+    """Weak scaling: every rank decodes its own batch of base.R requests (its own seeds)."""
+    return base.scaled(seed=base.seed + 7919 * rank)
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Maximum of a per-rank number over all ranks (the job's time is its slowest rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args):
@@ -265,15 +283,10 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        tt = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        return float(tt.item())
+    def max_ranks(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
-    base = wl.WORKLOADS[args.workload]
-    w = base.scaled(seed=base.seed + 7919 * rank)       # every rank: its own requests
+    w = rank_workload(wl.WORKLOADS[args.workload], rank)
     cores = len(os.sched_getaffinity(0))
     pool = None
     do_cpu = (not args.no_cpu_baseline) and rank == 0 and world == 1
@@ -330,7 +343,7 @@ def run_ours(args):
     st = dec.error()
     if st != ola.OLA_OK:
         raise RuntimeError(f"device error in the timed region: {ola.ola_strerror(st)}")
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms = max_ranks(e0.elapsed_time(e1))
     step_ms = np.array([[evs[k][t][0].elapsed_time(evs[k][t][1]) for t in range(w.T)]
                         for k in range(K)])
     per_launch_ms = step_ms.mean(axis=0)               # ola_step t, averaged over K
@@ -385,7 +398,7 @@ def run_ours(args):
                 decode(d2)
             b.record(stream)
             torch.cuda.synchronize()
-            mms = max_over_ranks(a.elapsed_time(b)) / reps
+            mms = max_ranks(a.elapsed_time(b)) / reps
             comps[name] = {"ms_per_step": mms, "value": world * units_per_step / (mms / 1e3),
                            "replay_tensor_speedup": mms / (ms / K)}
             d2.close()
@@ -413,7 +426,7 @@ def run_ours(args):
         t0 = time.perf_counter()
         for _ in range(args.e2e_steps):
             decode_host()
-        dt = max_over_ranks(time.perf_counter() - t0)
+        dt = max_ranks(time.perf_counter() - t0)
         result["e2e"] = {"value": world * units_per_step * args.e2e_steps / dt, "unit": UNIT,
                          "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                          "ms_per_step": 1e3 * dt / args.e2e_steps,
