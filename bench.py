@@ -69,7 +69,7 @@ def measured_peaks() -> dict:
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("ola_replay_tc.cu", "ola_plan.cu", "ola_device.cuh"):
+    for f in ("ola_replay_pos.cu", "ola_plan.cu", "ola_device.cuh"):
         h.update(open(os.path.join(ROOT, "linear_attention_beam_gdn_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -77,7 +77,7 @@ def kernel_source_hash() -> str:
 def recorded_traffic(workload: str):
     """DRAM bytes per launch of the replay kernel from the committed ncu summary, if it was
     taken on the current kernel source (else None)."""
-    p = os.path.join(ROOT, "profiles", "replay_tc_traffic.json")
+    p = os.path.join(ROOT, "profiles", "replay_pos_traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
@@ -104,7 +104,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -286,7 +286,10 @@ def run_ours(args):
     def max_ranks(x: float) -> float:
         return max_over_ranks(x, world, dev)
 
-    w = rank_workload(wl.WORKLOADS[args.workload], rank)
+    base = wl.WORKLOADS[args.workload]
+    if args.requests:
+        base = base.scaled(R=args.requests)
+    w = rank_workload(base, rank)
     cores = len(os.sched_getaffinity(0))
     pool = None
     do_cpu = (not args.no_cpu_baseline) and rank == 0 and world == 1
@@ -360,7 +363,7 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"],
                 "traffic": recorded_traffic(w.name),
-                "kernel": "ola_step (ola::plan_kernel + ola::replay_tc_kernel<128,128>)",
+                "kernel": "ola_step = ola::plan_kernel + ola::replay_pos_kernel<128,128,64>",
                 "algorithmic_bytes_per_decode": int(sum(bytes_t)),
                 "algorithmic_bytes_per_launch": [int(b) for b in bytes_t],
                 "launch_ms": [round(float(x), 4) for x in per_launch_ms],
@@ -458,7 +461,7 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="stress", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -466,6 +469,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--requests", type=int, default=0,
+                    help="override the workload's request count (profiling a smaller case)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warm-up raised to 3", file=sys.stderr)

@@ -172,8 +172,7 @@ replay_pos_kernel(const __grid_constant__ CUtensorMap tm_shi,
 
   // -------------------------------------------------------------------- phase 1
   // Round 1: the beams of this warp's positions and their parents' chains (both indexed by
-  // position). Round 2: q_t, k_t rows, g, beta, the chain's alphas. The rows that phases 2 and
-  // 3 will gather (ancestors' k_j and w_j, v) are prefetched into L2 as soon as known.
+  // position). Round 2: q_t, k_t rows, g, beta, the chain's alphas.
   int recs[PPW];
 #pragma unroll
   for (int jj = 0; jj < PPW; ++jj) {
@@ -194,29 +193,18 @@ replay_pos_kernel(const __grid_constant__ CUtensorMap tm_shi,
   }
   int rows[PPW];
   float al[PPW];
+  // record row of (step lane+1, request r, head h, beam 0): rows are this base + beam index
+  const int row_base = int(rec_index(a, lane < n_anc ? lane : 0, r, h, 0));
 #pragma unroll
   for (int jj = 0; jj < PPW; ++jj) {
     const bool vj = c0 + p0 + jj < a.B;
-    rows[jj] = int(rec_index(a, lane < n_anc ? lane : 0, r, h, recs[jj]));
+    rows[jj] = row_base + recs[jj];
     al[jj] = (vj && lane < n_anc) ? a.A[rows[jj]] : 1.f;
-    if (vj && lane < n_anc) {
-      const char* kr = reinterpret_cast<const char*>(
-          static_cast<const __nv_bfloat16*>(a.Kr) + size_t(rows[jj]) * DK);
-      const char* wr = reinterpret_cast<const char*>(a.W + size_t(rows[jj]) * DV);
-#pragma unroll
-      for (int c = 0; c < DK * 2; c += 128) prefetch_l2(kr + c);
-#pragma unroll
-      for (int c = 0; c < DV * 4; c += 128) prefetch_l2(wr + c);
-    }
   }
   float my_alpha = 0.f, my_beta = 0.f;
   if (lane < PPW && my_valid) {
     my_alpha = expf(a.g[my_io]);
     my_beta = a.beta[my_io];
-    const char* vr = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(a.v) +
-                                                   size_t(my_io) * DV);
-#pragma unroll
-    for (int c = 0; c < DV * 2; c += 128) prefetch_l2(vr + c);
   }
   KVec qv[PPW], kv[PPW];
 #pragma unroll
