@@ -22,6 +22,10 @@ cudaError_t launch_replay_pos(const StepArgs& a, const CUtensorMap& mhi, const C
 size_t replay_pos_smem(int d_k, int d_v, int T_max);
 bool replay_pos_supported(int d_k, int d_v);
 bool make_state_map(CUtensorMap* map, const void* base, int RH, int d_k, int d_v);
+bool replay_pipe_supported(int d_k, int d_v, int T_max);
+size_t replay_pipe_smem(int d_k, int T_max);
+cudaError_t launch_replay_pipe(const StepArgs& a, const void* S_hi, const void* S_lo,
+                               cudaStream_t stream);
 cudaError_t launch_split_state(const float* S, void* hi, void* lo, int RH, int d_k, int d_v,
                                cudaStream_t stream);
 }  // namespace ola
@@ -47,6 +51,7 @@ struct ola_ctx {
   int* pchain = nullptr;     // [R][B][T_max] parent chain by depth-first position
   int* err = nullptr;
   CUtensorMap m_hi, m_lo;
+  bool pipe = false;         // tensor path on the persistent pipelined kernel
   // staging buffers of ola_step_host (allocated on first use)
   void* st[7] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
   cudaStream_t last_stream = nullptr;
@@ -205,6 +210,8 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
   if (geom->path == OLA_PATH_REPLAY) {
     size_t smem = geom->math != OLA_MATH_TENSOR
                       ? replay_simt_smem(geom->d_k, geom->d_v, geom->T_max)
+                  : replay_pipe_supported(geom->d_k, geom->d_v, geom->T_max)
+                      ? replay_pipe_smem(geom->d_k, geom->T_max)
                   : replay_pos_supported(geom->d_k, geom->d_v)
                       ? replay_pos_smem(geom->d_k, geom->d_v, geom->T_max)
                       : replay_tc_smem(geom->d_k, geom->d_v, geom->B, geom->T_max);
@@ -243,6 +250,7 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
     if (e == cudaSuccess && (!make_state_map(&h->m_hi, h->S_hi, RH, geom->d_k, geom->d_v) ||
                              !make_state_map(&h->m_lo, h->S_lo, RH, geom->d_k, geom->d_v)))
       e = cudaErrorInvalidValue;
+    h->pipe = replay_pipe_supported(geom->d_k, geom->d_v, geom->T_max);
   }
   if (e != cudaSuccess) {
     ola_status rs = from_cuda(e);
@@ -269,6 +277,8 @@ ola_status ola_step(ola_handle h, const void* q, const void* k, const void* v, c
   cudaError_t e;
   if (h->g.path == OLA_PATH_FULLSTATE)
     e = launch_fullstate(a, h->g.in_dtype, st);
+  else if (h->g.math == OLA_MATH_TENSOR && h->pipe)
+    e = launch_replay_pipe(a, h->S_hi, h->S_lo, st);
   else if (h->g.math == OLA_MATH_TENSOR && replay_pos_supported(h->g.d_k, h->g.d_v))
     e = launch_replay_pos(a, h->m_hi, h->m_lo, st);
   else if (h->g.math == OLA_MATH_TENSOR)

@@ -25,8 +25,8 @@
 //            row appended; the parent's chain (record rows, alphas) into a per-beam table;
 //            k_t . q_t.
 //   MMA      warp 0 lane 0, once the S_ctx slices (TMA at CTA start) and the A tiles are in.
-//   phase 2  k_j . k_t and k_j . q_t for every ancestor (4-lane groups, 8 beams at once), then
-//            the decay pass.
+//   phase 2  k_j . k_t and k_j . q_t for every ancestor on warp-level tensor-core MMA
+//            (16 (beam, ancestor) rows x 8 beams per m16n8k16), then the decay pass.
 //   D        tensor memory -> shared memory transposed to beam-major rows, reusing the space
 //            of the S and A tiles (XOR-swizzled by row: conflict-free both ways).
 //   phase 3  per beam: Y rows, ancestors' w_j rows, v row -> u, w_t, o_t -> o and w_t rows.
@@ -296,55 +296,57 @@ replay_pos_kernel(const __grid_constant__ CUtensorMap tm_shi,
   }
 
   // -------------------------------------------------------------------- phase 2: dots
-  // Lane groups: lane (j, g) = (lane / 4, lane % 4) holds d_k elements [g DK/4, (g+1) DK/4) of
-  // position j of this warp (k_t, q_t re-read from the A tiles); per ancestor it loads the
-  // same slice of k_j and the group sums over its 4 lanes. The 8 positions go in parallel,
-  // 4 ancestors' loads in flight per round.
+  // Warp-level tensor-core MMA (m16n8k16, bf16 in, fp32 accumulate): the 16 rows of A are the
+  // keys of ancestors s0 (rows 0-7) and s0+1 (rows 8-15) of the warp's 8 positions, the 8
+  // columns of B are those positions' k_t (then q_t). Only the diagonal D[j][j], D[8+j][j] is
+  // used. The k index is permuted consistently in A and B (the dot product is a sum) so that
+  // lane (g, c) of each fragment reads whole 16-byte chunks: chunk m of a row = elements
+  // [32 m + 8 c, +8), which feed virtual k-steps 2m and 2m+1.
   {
-    constexpr int GE = DK / 4;                       // elements per lane
-    constexpr int GC = GE / 8;                       // 16-byte chunks per lane
-    const int j = lane >> 2, g = lane & 3;
-    const int pn = p0 + j;
-    uint4 xq[GC], xk[GC];
+    const int gq = lane >> 2, cq4 = lane & 3;
+    const int pn = p0 + gq;
+    uint4 xk[DK / 32], xq[DK / 32];
 #pragma unroll
-    for (int c = 0; c < GC; ++c) {
-      const int e = g * GE + 8 * c;
+    for (int m = 0; m < DK / 32; ++m) {
+      const int e = 32 * m + 8 * cq4;
       const int ks = e / 64, ch = (e % 64) / 8;
-      xq[c] = *reinterpret_cast<const uint4*>(x_tile(ks, 0) + pn * 128 + ((ch ^ (pn & 7)) * 16));
-      xk[c] = *reinterpret_cast<const uint4*>(x_tile(ks, 1) + pn * 128 + ((ch ^ (pn & 7)) * 16));
+      xk[m] = *reinterpret_cast<const uint4*>(x_tile(ks, 1) + pn * 128 + ((ch ^ (pn & 7)) * 16));
+      xq[m] = *reinterpret_cast<const uint4*>(x_tile(ks, 0) + pn * 128 + ((ch ^ (pn & 7)) * 16));
     }
     const __nv_bfloat16* krec = static_cast<const __nv_bfloat16*>(a.Kr);
-    for (int s0 = 0; s0 < n_anc; s0 += 4) {
-      uint4 kj[4][GC];
+    constexpr int NP = 2;                          // ancestor pairs per round (4 rows in flight)
+    for (int s0 = 0; s0 < n_anc; s0 += 2 * NP) {
+      uint4 kr[2 * NP][DK / 32];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const bool in = s0 + m < n_anc;
-        const int row = tab[pn * TA + (in ? s0 + m : 0)].row;
-        const uint4* src = reinterpret_cast<const uint4*>(krec + size_t(row) * DK + g * GE);
+      for (int i = 0; i < 2 * NP; ++i) {
+        const int s = s0 + i < n_anc ? s0 + i : s0;
+        const uint4* src =
+            reinterpret_cast<const uint4*>(krec + size_t(tab[pn * TA + s].row) * DK + 8 * cq4);
 #pragma unroll
-        for (int c = 0; c < GC; ++c) kj[m][c] = in ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        for (int m = 0; m < DK / 32; ++m) kr[i][m] = src[4 * m];
       }
-      float dk[4], dq[4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        dk[m] = 0.f;
-        dq[m] = 0.f;
+      for (int pr = 0; pr < NP; ++pr) {
+        const uint4* ka = kr[2 * pr];
+        const uint4* kb = kr[2 * pr + 1];
+        float dk[4] = {0.f, 0.f, 0.f, 0.f}, dq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < GC; ++c) {
-          dk[m] = dot_bf16<4>(kj[m][c], xk[c], dk[m]);
-          dq[m] = dot_bf16<4>(kj[m][c], xq[c], dq[m]);
+        for (int m = 0; m < DK / 32; ++m) {
+          mma_16816_bf16(dk, ka[m].x, kb[m].x, ka[m].y, kb[m].y, xk[m].x, xk[m].y);
+          mma_16816_bf16(dq, ka[m].x, kb[m].x, ka[m].y, kb[m].y, xq[m].x, xq[m].y);
+          mma_16816_bf16(dk, ka[m].z, kb[m].z, ka[m].w, kb[m].w, xk[m].z, xk[m].w);
+          mma_16816_bf16(dq, ka[m].z, kb[m].z, ka[m].w, kb[m].w, xq[m].z, xq[m].w);
         }
-        dk[m] += __shfl_xor_sync(0xffffffffu, dk[m], 1);
-        dq[m] += __shfl_xor_sync(0xffffffffu, dq[m], 1);
-        dk[m] += __shfl_xor_sync(0xffffffffu, dk[m], 2);
-        dq[m] += __shfl_xor_sync(0xffffffffu, dq[m], 2);
-      }
-      if (g == 0) {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          if (s0 + m < n_anc) {
-            tab[pn * TA + s0 + m].cu = dk[m];
-            tab[pn * TA + s0 + m].cq = dq[m];
+        const int s = s0 + 2 * pr;
+        if (cq4 == (gq >> 1)) {                      // this lane holds column gq = position gq
+          const int o = gq & 1;
+          if (s < n_anc) {
+            tab[pn * TA + s].cu = dk[o];
+            tab[pn * TA + s].cq = dq[o];
+          }
+          if (s + 1 < n_anc) {
+            tab[pn * TA + s + 1].cu = dk[2 + o];
+            tab[pn * TA + s + 1].cq = dq[2 + o];
           }
         }
       }
