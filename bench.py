@@ -69,7 +69,7 @@ def measured_peaks() -> dict:
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("ola_replay_pipe.cu", "ola_plan.cu", "ola_device.cuh"):
+    for f in ("ola_replay_mma.cu", "ola_plan.cu", "ola_device.cuh"):
         h.update(open(os.path.join(ROOT, "linear_attention_beam_gdn_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -77,7 +77,7 @@ def kernel_source_hash() -> str:
 def recorded_traffic(workload: str):
     """DRAM bytes per launch of the replay kernel from the committed ncu summary, if it was
     taken on the current kernel source (else None)."""
-    p = os.path.join(ROOT, "profiles", "replay_pipe_traffic.json")
+    p = os.path.join(ROOT, "profiles", "replay_mma_traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
@@ -363,7 +363,7 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"],
                 "traffic": recorded_traffic(w.name),
-                "kernel": "ola_step = ola::plan_kernel + ola::replay_pipe_kernel<128>",
+                "kernel": "ola_step = ola::plan_units_kernel + ola::replay_mma_kernel<128>",
                 "algorithmic_bytes_per_decode": int(sum(bytes_t)),
                 "algorithmic_bytes_per_launch": [int(b) for b in bytes_t],
                 "launch_ms": [round(float(x), 4) for x in per_launch_ms],

@@ -26,6 +26,14 @@ bool replay_pipe_supported(int d_k, int d_v, int T_max);
 size_t replay_pipe_smem(int d_k, int T_max);
 cudaError_t launch_replay_pipe(const StepArgs& a, const void* S_hi, const void* S_lo,
                                cudaStream_t stream);
+bool replay_mma_supported(int d_k, int d_v, int B, int T_max);
+size_t replay_mma_smem(int d_k);
+size_t plan_units_smem(int B, int T_max);
+cudaError_t launch_replay_mma(const StepArgs& a, const UnitPlan& up, const void* S_hi,
+                              const void* S_lo, const CUtensorMap& mkr, const CUtensorMap& mw,
+                              cudaStream_t stream);
+bool make_record_maps(CUtensorMap* mkr, CUtensorMap* mw, const void* Kr, const void* W,
+                      uint64_t n_rec, int d_k, int d_v);
 cudaError_t launch_split_state(const float* S, void* hi, void* lo, int RH, int d_k, int d_v,
                                cudaStream_t stream);
 }  // namespace ola
@@ -51,7 +59,10 @@ struct ola_ctx {
   int* pchain = nullptr;     // [R][B][T_max] parent chain by depth-first position
   int* err = nullptr;
   CUtensorMap m_hi, m_lo;
+  CUtensorMap m_kr, m_w;     // record row maps of the mma kernel
   bool pipe = false;         // tensor path on the persistent pipelined kernel
+  bool mma = false;          // tensor path with the replay accumulation on tensor cores
+  UnitPlan up{};             // units of work of the mma kernel (rewritten every step)
   // staging buffers of ola_step_host (allocated on first use)
   void* st[7] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
   cudaStream_t last_stream = nullptr;
@@ -83,10 +94,17 @@ ola_status validate(const ola_geometry* g) {
 
 struct Sizes {
   size_t S, S_split, W, Kr, A, C, FS, perm, rank, pchain, err;
+  size_t ucnt, uoff, urec, upos, counter;   // mma path only
   size_t total() const {
-    return S + 2 * S_split + W + Kr + A + C + 2 * FS + perm + rank + pchain + err;
+    return S + 2 * S_split + W + Kr + A + C + 2 * FS + perm + rank + pchain + err + ucnt + uoff +
+           urec + upos + counter;
   }
 };
+
+bool uses_mma(const ola_geometry* g) {
+  return g->math == OLA_MATH_TENSOR && g->path == OLA_PATH_REPLAY &&
+         replay_mma_supported(g->d_k, g->d_v, g->B, g->T_max);
+}
 
 Sizes sizes_of(const ola_geometry* g) {
   Sizes z{};
@@ -104,6 +122,14 @@ Sizes sizes_of(const ola_geometry* g) {
   z.rank = g->math == OLA_MATH_TENSOR ? 2 * R * B * 4 : 0;
   z.pchain = g->math == OLA_MATH_TENSOR ? R * B * T * 4 : 0;
   z.err = 16;
+  if (uses_mma(g)) {
+    z.ucnt = R * 4;
+    z.uoff = (R + 1) * 4;
+    z.urec = R * B * size_t(kUnitRecInts) * 4;   // at most B units per request
+    z.upos = R * B * 16;
+    z.counter = 16;
+    z.pchain = 0;
+  }
   return z;
 }
 
@@ -124,8 +150,9 @@ cudaError_t dev_alloc(T** p, size_t bytes) {
 }
 
 void free_all(ola_ctx* h) {
-  void* ptrs[] = {h->S,     h->S_hi,  h->S_lo, h->W,    h->Kr,  h->A,
-                  h->C,     h->FS[0], h->FS[1], h->perm, h->rank, h->pchain, h->err};
+  void* ptrs[] = {h->S,     h->S_hi,  h->S_lo,   h->W,       h->Kr,     h->A,
+                  h->C,     h->FS[0], h->FS[1],  h->perm,    h->rank,   h->pchain,
+                  h->err,   h->up.ucnt, h->up.uoff, h->up.urec, h->up.upos, h->up.counter};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (void* p : h->st)
@@ -210,12 +237,16 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
   if (geom->path == OLA_PATH_REPLAY) {
     size_t smem = geom->math != OLA_MATH_TENSOR
                       ? replay_simt_smem(geom->d_k, geom->d_v, geom->T_max)
+                  : uses_mma(geom) ? replay_mma_smem(geom->d_k)
                   : replay_pipe_supported(geom->d_k, geom->d_v, geom->T_max)
                       ? replay_pipe_smem(geom->d_k, geom->T_max)
                   : replay_pos_supported(geom->d_k, geom->d_v)
                       ? replay_pos_smem(geom->d_k, geom->d_v, geom->T_max)
                       : replay_tc_smem(geom->d_k, geom->d_v, geom->B, geom->T_max);
     if (smem > size_t(prop.sharedMemPerBlockOptin)) return OLA_ERR_UNSUPPORTED;
+    if (uses_mma(geom) &&
+        plan_units_smem(geom->B, geom->T_max) > size_t(prop.sharedMemPerBlockOptin))
+      return OLA_ERR_UNSUPPORTED;
   }
 
   ola_ctx* h = new (std::nothrow) ola_ctx();
@@ -241,6 +272,13 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
   if (e == cudaSuccess) e = dev_alloc(&h->rank, z.rank);
   if (e == cudaSuccess) e = dev_alloc(&h->pchain, z.pchain);
   if (e == cudaSuccess) e = dev_alloc(&h->err, z.err);
+  if (e == cudaSuccess) e = dev_alloc(&h->up.ucnt, z.ucnt);
+  if (e == cudaSuccess) e = dev_alloc(&h->up.uoff, z.uoff);
+  if (e == cudaSuccess) e = dev_alloc(&h->up.urec, z.urec);
+  if (e == cudaSuccess) e = dev_alloc(&h->up.upos, z.upos);
+  if (e == cudaSuccess) e = dev_alloc(&h->up.counter, z.counter);
+  if (e == cudaSuccess && z.counter) e = cudaMemsetAsync(h->up.counter, 0, z.counter, st);
+  h->up.maxU = geom->B;
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->S, S_ctx, z.S, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, z.err, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->C, 0, z.C, st);
@@ -250,7 +288,12 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
     if (e == cudaSuccess && (!make_state_map(&h->m_hi, h->S_hi, RH, geom->d_k, geom->d_v) ||
                              !make_state_map(&h->m_lo, h->S_lo, RH, geom->d_k, geom->d_v)))
       e = cudaErrorInvalidValue;
-    h->pipe = replay_pipe_supported(geom->d_k, geom->d_v, geom->T_max);
+    h->mma = uses_mma(geom);
+    h->pipe = !h->mma && replay_pipe_supported(geom->d_k, geom->d_v, geom->T_max);
+    const uint64_t n_rec = uint64_t(geom->T_max) * geom->R * geom->H * geom->B;
+    if (e == cudaSuccess && h->mma &&
+        !make_record_maps(&h->m_kr, &h->m_w, h->Kr, h->W, n_rec, geom->d_k, geom->d_v))
+      e = cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) {
     ola_status rs = from_cuda(e);
@@ -277,6 +320,8 @@ ola_status ola_step(ola_handle h, const void* q, const void* k, const void* v, c
   cudaError_t e;
   if (h->g.path == OLA_PATH_FULLSTATE)
     e = launch_fullstate(a, h->g.in_dtype, st);
+  else if (h->g.math == OLA_MATH_TENSOR && h->mma)
+    e = launch_replay_mma(a, h->up, h->S_hi, h->S_lo, h->m_kr, h->m_w, st);
   else if (h->g.math == OLA_MATH_TENSOR && h->pipe)
     e = launch_replay_pipe(a, h->S_hi, h->S_lo, st);
   else if (h->g.math == OLA_MATH_TENSOR && replay_pos_supported(h->g.d_k, h->g.d_v))

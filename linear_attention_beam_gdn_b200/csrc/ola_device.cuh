@@ -45,6 +45,23 @@ struct StepArgs {
   int* err;                     // device error word: [0] code, [1] detail, [2] step
 };
 
+// Units of work of the tensor-core replay kernel, written each step by plan_units_kernel
+// (ola_plan.cu): at most kUnitPos consecutive depth-first positions of one request whose
+// parent chains reach at most kUnitAnc distinct records.
+constexpr int kUnitPos = 32;
+constexpr int kUnitAnc = 48;
+constexpr int kUnitRecInts = 96;
+
+struct UnitPlan {
+  int* ucnt;          // [R] units of each request
+  int* uoff;          // [R + 1] exclusive prefix sum of ucnt
+  int* urec;          // [R][maxU][kUnitRecInts]
+  uint8_t* upos;      // [R][B][16]
+  unsigned* counter;  // CTAs finished (reset to 0 by the last one)
+  int maxU;           // units per request at most
+};
+
+
 __host__ __device__ __forceinline__ size_t rec_index(const StepArgs& a, int slot, int r, int h,
                                                      int b) {
   return ((size_t(slot) * a.R + r) * a.H + h) * size_t(a.B) + b;
@@ -107,6 +124,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// First 1024-byte aligned byte of the dynamic shared memory. The offset is computed from the
+// shared-window address but applied by pointer arithmetic on the __shared__ array, so the
+// compiler still knows the result points into shared memory (an integer round trip through
+// uintptr_t would turn every access through it into a generic load or store).
+__device__ __forceinline__ unsigned char* align_smem_1024(unsigned char* base) {
+  return base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                : "memory");
@@ -158,6 +183,54 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// ------------------------------------------------------------------ cp.async (Ampere-style)
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// 16-byte global -> shared copy, cached in L2 only; both addresses 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread has issued so far has landed (counts as one
+// of the barrier's expected arrivals).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Dot product of 8 bf16 pairs (two 16-byte chunks), fp32 products and sum.
+__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
+  const uint32_t x[4] = {a.x, a.y, a.z, a.w}, y[4] = {b.x, b.y, b.z, b.w};
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    s = fmaf(__uint_as_float(x[i] << 16), __uint_as_float(y[i] << 16), s);
+    s = fmaf(__uint_as_float(x[i] & 0xffff0000u), __uint_as_float(y[i] & 0xffff0000u), s);
+  }
+  return s;
+}
+
+// Barrier over `count` threads (a multiple of 32) of the CTA, id 1..15 (0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Four 8x8 b16 matrices from shared memory (lane l gives the row address of matrix l / 8).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+
 // ------------------------------------------------------------------ TMA (no multicast)
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
@@ -179,15 +252,16 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Row gather (sm_100a): rows y0..y3 of a 2-D tensor map whose box is one row high, columns from
-// x, written to shared memory one after another (4 x the box's row bytes from dst). With the
-// 128-byte swizzle the chunk permutation follows the shared-memory address, so a gather into
-// row 4m of a 1024-byte aligned tile lands as rows 4m..4m+3 of the canonical swizzled layout.
+// Row gather (sm_100a): rows y0..y3 of a 2-D tensor map whose box is one row high (64 bf16
+// columns from x, x a multiple of 64), written to shared memory as four consecutive 128-byte
+// rows from dst (dst 128-byte aligned; with the 128-byte swizzle the chunk order follows the
+// shared-memory address, so a 1024-byte aligned tile filled four rows at a time is the
+// canonical swizzled layout). Completion counted on `bar` as 512 transaction bytes.
 __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y0, int y1, int y2, int y3) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      ".cta_group::1 [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
       "r"(smem_u32(bar))
       : "memory");
@@ -319,6 +393,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (uint32_t(M >> 4) << 24);                // M / 16
 }
 
+// Shared-memory matrix descriptor, MN-major operand with the 128-byte swizzle: each 128-byte
+// row holds 64 consecutive M (or N) elements of one K index, 8 rows (8 K) form a 1024-byte
+// atom; `lbo` = byte distance between 64-element blocks along M/N, `sbo` = byte distance
+// between groups of 8 K.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t lbo,
+                                                       uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((smem_addr & 0x3FFFFu) >> 4);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, A MN-major, B K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_amn(int M, int N) {
+  return idesc_bf16_f32(M, N) | (1u << 15);
+}
+
 // Two loads of 32 lanes x 8 consecutive 32-bit columns from tensor memory (one lane per
 // thread) followed by the wait, in one asm statement so that no instruction can read the
 // destination registers before the asynchronous loads have landed.
@@ -339,6 +433,89 @@ __device__ __forceinline__ void tmem_ld8x2(uint32_t ta, uint32_t tb, float (&xa)
     xa[j] = __uint_as_float(r[j]);
     xb[j] = __uint_as_float(r[8 + j]);
   }
+}
+
+// Four loads of 32 lanes x 8 consecutive 32-bit columns, then the wait (one asm statement).
+__device__ __forceinline__ void tmem_ld8x4(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3,
+                                           float (&x0)[8], float (&x1)[8], float (&x2)[8],
+                                           float (&x3)[8]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8, %9, %10, %11, %12, %13, %14, %15}, [%33];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16, %17, %18, %19, %20, %21, %22, %23}, [%34];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%24, %25, %26, %27, %28, %29, %30, %31}, [%35];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(t0), "r"(t1), "r"(t2), "r"(t3)
+      : "memory");
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    x0[j] = __uint_as_float(r[j]);
+    x1[j] = __uint_as_float(r[8 + j]);
+    x2[j] = __uint_as_float(r[16 + j]);
+    x3[j] = __uint_as_float(r[24 + j]);
+  }
+}
+
+// One load of 32 lanes x 16 consecutive 32-bit columns, then the wait.
+__device__ __forceinline__ void tmem_ld16(uint32_t t, float (&x)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(t)
+      : "memory");
+#pragma unroll
+  for (int j = 0; j < 16; ++j) x[j] = __uint_as_float(r[j]);
+}
+
+// Four loads of 32 lanes x 16 consecutive 32-bit columns, then the wait, in one asm statement
+// (no instruction can read the destination registers before the loads have landed).
+__device__ __forceinline__ void tmem_ld16x4(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3,
+                                            float (&x0)[16], float (&x1)[16], float (&x2)[16],
+                                            float (&x3)[16]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%65];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47}, [%66];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%67];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(t0), "r"(t1), "r"(t2), "r"(t3)
+      : "memory");
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    x0[j] = __uint_as_float(r[j]);
+    x1[j] = __uint_as_float(r[16 + j]);
+    x2[j] = __uint_as_float(r[32 + j]);
+    x3[j] = __uint_as_float(r[48 + j]);
+  }
+}
+
+// Three loads of 32 lanes x 16 consecutive 32-bit columns, then the wait.
+__device__ __forceinline__ void tmem_ld16x3(uint32_t t0, uint32_t t1, uint32_t t2, float (&x)[48]) {
+  uint32_t r[48];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%48];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%49];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47}, [%50];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47])
+      : "r"(t0), "r"(t1), "r"(t2)
+      : "memory");
+#pragma unroll
+  for (int j = 0; j < 48; ++j) x[j] = __uint_as_float(r[j]);
 }
 
 }  // namespace ola

@@ -68,4 +68,254 @@ cudaError_t launch_plan(const StepArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------- units of work
+
+// Depth-first positions cut into units for the tensor-core replay kernel (ola_replay_mma.cu).
+//
+// A unit is a run of at most kUnitPos consecutive depth-first positions of one request whose
+// parent chains reach at most kUnitAnc distinct records. In depth-first order every record's
+// descendants are contiguous, so within a chain slot the records of consecutive positions are
+// equal or new, and the distinct records of a unit are the slot-wise changes. Units are made of
+// whole sibling groups where they fit (see the cut below).
+//
+// For every unit the kernel writes one record of kUnitRecInts ints:
+//   [0] start | n_pos << 16, [1] U (distinct records), [4 + p] beam at position start + p,
+//   [36 + u] (slot << 16) | beam of distinct record u (slot order, then position order),
+// and for every position p, upos[r][p][s] = index u of the record in chain slot s. It also
+// writes the chain rows of the new beams (C[t-1][r][b] = parent's chain, then b), the number
+// of units of each request and, in the last CTA to finish, their exclusive prefix sum.
+size_t plan_units_smem(int B, int T_max) {
+  const int Bp = (B + 3) & ~3, TA = T_max > 1 ? T_max - 1 : 1;
+  // keys, parents, perm, chains, change masks, unit of position, unit start/size/U, counts,
+  // sibling-group starts and sizes, scratch
+  return sizeof(int) * (size_t(Bp) + B + B + size_t(B) * TA + B + B + 3 * size_t(B) +
+                        size_t(B) * TA + 2 * size_t(B) + 64);
+}
+
+__global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up) {
+  extern __shared__ int sm[];
+  const int r = blockIdx.x, B = a.B, Bp = (B + 3) & ~3;
+  const int n_anc = a.t - 1, TA = a.T_max > 1 ? a.T_max - 1 : 1;
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  int* keys = sm;                 // [Bp]
+  int* pbuf = keys + Bp;          // [B] clamped parent of beam b
+  int* sperm = pbuf + B;          // [B] beam at position
+  int* spch = sperm + B;          // [B][TA] parent chain by position
+  int* fnew = spch + B * TA;      // [B] slots where the record differs from the position before
+  int* uop = fnew + B;            // [B] unit of position
+  int* ustart = uop + B;          // [B]
+  int* un = ustart + B;           // [B]
+  int* uU = un + B;               // [B]
+  int* sdist = uU + B;            // [B][TA] distinct records per (unit, slot)
+  int* gst = sdist + B * TA;      // [B] start of each sibling group
+  int* gsz = gst + B;             // [B] its size
+  int* misc = gsz + B;            // [0] unit count, [1] last-CTA flag, [2] groups, [32..] scratch
+
+  // depth-first order: stable sort of the beams by their parent's position (ola_plan.cu above)
+  for (int b = tid; b < Bp; b += nt) {
+    int key = INT_MAX;
+    if (b < B) {
+      const int p = checked_parent(a, r, b);
+      key = (a.t == 1) ? 0 : a.rank_prev[size_t(r) * B + p];
+      pbuf[b] = p;
+    }
+    keys[b] = key;
+  }
+  __syncthreads();
+  const int4* k4 = reinterpret_cast<const int4*>(keys);
+  for (int b = tid; b < B; b += nt) {
+    const int k = keys[b];
+    int pos = 0;
+    for (int j = 0; j < Bp / 4; ++j) {
+      const int4 kk = k4[j];
+      const int b2 = 4 * j;
+      pos += (kk.x < k) | ((kk.x == k) & (b2 + 0 < b));
+      pos += (kk.y < k) | ((kk.y == k) & (b2 + 1 < b));
+      pos += (kk.z < k) | ((kk.z == k) & (b2 + 2 < b));
+      pos += (kk.w < k) | ((kk.w == k) & (b2 + 3 < b));
+    }
+    a.perm[size_t(r) * B + pos] = b;
+    a.rank_cur[size_t(r) * B + b] = pos;
+    sperm[pos] = b;
+  }
+  __syncthreads();
+  // parent chains by position; chain rows of the new beams
+  for (int x = tid; x < B * n_anc; x += nt) {
+    const int pos = x / n_anc, s = x % n_anc;
+    const int b = sperm[pos];
+    const int c = a.C[chain_row(a, a.t - 2, r, pbuf[b]) + s];
+    spch[pos * TA + s] = c;
+    a.C[chain_row(a, a.t - 1, r, b) + s] = c;
+  }
+  for (int pos = tid; pos < B; pos += nt) a.C[chain_row(a, a.t - 1, r, sperm[pos]) + n_anc] = sperm[pos];
+  __syncthreads();
+  for (int pos = tid; pos < B; pos += nt) {
+    int m = 0;
+    for (int s = 0; s < n_anc; ++s)
+      if (pos == 0 || spch[pos * TA + s] != spch[(pos - 1) * TA + s]) m |= 1 << s;
+    fnew[pos] = m;
+  }
+  __syncthreads();
+  // sibling groups (runs of positions with the same parent): numbered by a block-wide scan
+  {
+    int carry = 0;
+    for (int base = 0; base < B; base += nt) {
+      const int pos = base + tid;
+      const int f = (pos < B && (pos == 0 || keys[sperm[pos]] != keys[sperm[pos - 1]])) ? 1 : 0;
+      int x = f;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, off);
+        if (lane >= off) x += y;
+      }
+      if (lane == 31) misc[32 + warp] = x;
+      __syncthreads();
+      int before = 0, tot = 0;
+      for (int w2 = 0; w2 < nt / 32; ++w2) {
+        if (w2 < warp) before += misc[32 + w2];
+        tot += misc[32 + w2];
+      }
+      if (f) gst[carry + before + x - 1] = pos;
+      carry += tot;
+      __syncthreads();
+    }
+    if (tid == 0) misc[2] = carry;
+    __syncthreads();
+    for (int g = tid; g < carry; g += nt) gsz[g] = (g + 1 < carry ? gst[g + 1] : B) - gst[g];
+  }
+  __syncthreads();
+  // units (one warp). Beams with the same parent have the same chain, and their outputs must not
+  // depend on how the beams are cut into units: a unit holds whole sibling groups of at most
+  // kUnitPos positions while its distinct records stay <= kUnitAnc (greedy, left to right);
+  // a larger group is cut into chunks of kUnitPos positions, each a unit of its own, so that
+  // every chunk lists the chain's records in the same order (record u = chain slot u).
+  if (warp == 0) {
+    const int ng = misc[2];
+    int g0 = 0, k = 0;
+    while (g0 < ng) {
+      const int gs0 = gst[g0], sz0 = gsz[g0];
+      if (sz0 > kUnitPos) {
+        for (int off = 0; off < sz0; off += kUnitPos) {
+          const int n = min(kUnitPos, sz0 - off);
+          if (lane == 0) {
+            ustart[k] = gs0 + off;
+            un[k] = n;
+            uU[k] = n_anc;
+          }
+          if (lane < n) uop[gs0 + off + lane] = k;
+          ++k;
+        }
+        ++g0;
+        continue;
+      }
+      const int g = g0 + lane;
+      const bool gv = g < ng;
+      int S = gv ? gsz[g] : (1 << 20);
+      int C = gv ? (lane == 0 ? n_anc : __popc(fnew[gst[g]])) : (1 << 20);
+      const unsigned bad = __ballot_sync(kFull, !gv || S > kUnitPos);
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int ys = __shfl_up_sync(kFull, S, off), yc = __shfl_up_sync(kFull, C, off);
+        if (lane >= off) {
+          S += ys;
+          C += yc;
+        }
+      }
+      const int firstbad = bad ? __ffs(bad) - 1 : 32;
+      // S, C grow with the lane, so the accepted lanes are a prefix; lane 0 always fits
+      const unsigned m = __ballot_sync(kFull, lane < firstbad && S <= kUnitPos && C <= kUnitAnc);
+      const int ngr = __popc(m);
+      const int n = __shfl_sync(kFull, S, ngr - 1), U = __shfl_sync(kFull, C, ngr - 1);
+      if (lane == 0) {
+        ustart[k] = gs0;
+        un[k] = n;
+        uU[k] = U;
+      }
+      if (lane < n) uop[gs0 + lane] = k;
+      ++k;
+      g0 += ngr;
+    }
+    if (lane == 0) misc[0] = k;
+  }
+  __syncthreads();
+  const int nu = misc[0];
+  int* rec_r = up.urec + size_t(r) * up.maxU * kUnitRecInts;
+  for (int x = tid; x < nu * n_anc; x += nt) {     // distinct records per (unit, slot)
+    const int k = x / n_anc, s = x % n_anc;
+    int cnt = 1;
+    for (int j = 1; j < un[k]; ++j) cnt += (fnew[ustart[k] + j] >> s) & 1;
+    sdist[k * TA + s] = cnt;
+  }
+  __syncthreads();
+  for (int x = tid; x < nu * n_anc; x += nt) {     // record list and per-position indices
+    const int k = x / n_anc, s = x % n_anc;
+    int base = 0;
+    for (int s2 = 0; s2 < s; ++s2) base += sdist[k * TA + s2];
+    int* rk = rec_r + size_t(k) * kUnitRecInts;
+    int c = 0;
+    for (int j = 0; j < un[k]; ++j) {
+      const int pos = ustart[k] + j;
+      if (j == 0 || ((fnew[pos] >> s) & 1)) {
+        rk[36 + base + c] = (s << 16) | spch[pos * TA + s];
+        ++c;
+      }
+      up.upos[(size_t(r) * B + pos) * 16 + s] = uint8_t(base + c - 1);
+    }
+  }
+  for (int k = tid; k < nu; k += nt) {
+    int* rk = rec_r + size_t(k) * kUnitRecInts;
+    rk[0] = ustart[k] | (un[k] << 16);
+    rk[1] = n_anc > 0 ? uU[k] : 0;
+  }
+  for (int pos = tid; pos < B; pos += nt) {
+    const int k = uop[pos];
+    rec_r[size_t(k) * kUnitRecInts + 4 + (pos - ustart[k])] = sperm[pos];
+  }
+  // unit counts; the last CTA to finish writes the prefix sums and resets the counter
+  if (tid == 0) {
+    up.ucnt[r] = nu;
+    __threadfence();
+    const unsigned ticket = atomicAdd(up.counter, 1u);
+    misc[1] = ticket == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (misc[1]) {
+    __threadfence();
+    int carry = 0;
+    int* wsum = misc + 32;
+    for (int base = 0; base < a.R; base += nt) {
+      const int v = base + tid < a.R ? __ldcg(up.ucnt + base + tid) : 0;
+      int x = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, off);
+        if (lane >= off) x += y;
+      }
+      if (lane == 31) wsum[warp] = x;
+      __syncthreads();
+      int before = 0, total = 0;
+      for (int w = 0; w < nt / 32; ++w) {
+        if (w < warp) before += wsum[w];
+        total += wsum[w];
+      }
+      if (base + tid < a.R) up.uoff[base + tid] = carry + before + x - v;
+      carry += total;
+      __syncthreads();
+    }
+    if (tid == 0) {
+      up.uoff[a.R] = carry;
+      *up.counter = 0u;
+    }
+  }
+}
+
+cudaError_t launch_plan_units(const StepArgs& a, const UnitPlan& up, cudaStream_t stream) {
+  const size_t smem = plan_units_smem(a.B, a.T_max);
+  cudaError_t e = cudaFuncSetAttribute(plan_units_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  plan_units_kernel<<<a.R, 512, smem, stream>>>(a, up);
+  return cudaGetLastError();
+}
+
 }  // namespace ola

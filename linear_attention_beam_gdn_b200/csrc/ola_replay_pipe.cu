@@ -82,35 +82,6 @@ __host__ __device__ inline PipeLayout pipe_layout(int d_k, int T_max) {
   return L;
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
-               : "memory");
-}
-
-// Arrive on `bar` once every cp.async this thread has issued so far has landed (counts as one
-// of the barrier's expected arrivals).
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
-  const uint32_t x[4] = {a.x, a.y, a.z, a.w}, y[4] = {b.x, b.y, b.z, b.w};
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    s = fmaf(__uint_as_float(x[i] << 16), __uint_as_float(y[i] << 16), s);
-    s = fmaf(__uint_as_float(x[i] & 0xffff0000u), __uint_as_float(y[i] & 0xffff0000u), s);
-  }
-  return s;
-}
-
-constexpr unsigned kFull = 0xffffffffu;
 
 template <int DK>
 __global__ void __launch_bounds__(kPipeWarps * 32, 1)
@@ -121,8 +92,7 @@ replay_pipe_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* 
   constexpr int CR = DK / 8;       // 16-byte chunks of a key row
   constexpr int RPI = 32 / CR;     // key rows copied per warp instruction
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem = align_smem_1024(smem_raw);
   const PipeLayout L = pipe_layout(DK, a.T_max);
   const int TA = L.TA;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);

@@ -121,8 +121,7 @@ replay_pos_kernel(const __grid_constant__ CUtensorMap tm_shi,
   static_assert(DK <= 128 && DV <= 128 && EPL >= 2 && VPL >= 2, "geometry");
 
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem = align_smem_1024(smem_raw);
   const PosLayout L = pos_layout(DK, DV, a.T_max, NB);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);   // [2]
   uint64_t* done = full + 2;

@@ -108,8 +108,7 @@ replay_tc_kernel(const __grid_constant__ CUtensorMap tm_shi,
   static_assert(CTRL || tc_resident(DK, DV), "resident variant needs d_k, d_v <= 128");
 
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem = align_smem_1024(smem_raw);
   const TcLayout L = tc_layout(DK, DV, NB, a.T_max);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);   // [4]
   uint64_t* empty = full + 4;                                        // [2]
@@ -447,6 +446,22 @@ bool make_state_map(CUtensorMap* map, const void* base, int RH, int d_k, int d_v
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
             box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// Rows of a 2-D bf16 matrix [rows][cols] (row stride row_bytes) for row gathers: box of 64
+// columns x 1 row, 128-byte swizzle (tile::gather4 loads four rows per instruction).
+bool make_rows_map(CUtensorMap* map, const void* base, uint64_t rows, int cols,
+                   uint64_t row_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(row_bytes)};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
 

@@ -68,11 +68,22 @@ def test_workspace_bytes_formula(L):
     gf = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, path=ola.OLA_PATH_FULLSTATE)
     expect_fs = R * H * dv * dk * 4 + 2 * R * H * B * dv * dk * 4 + T * R * B * T * 4 + 16
     assert ola.ola_workspace_bytes(gf) == expect_fs
+    # tensor path, d_v = 128: unit plan buffers (counts, prefix, unit records, per-position
+    # record indices, a counter) instead of the parent-chain table
     gt = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, in_dtype=ola.OLA_BF16,
                math=ola.OLA_MATH_TENSOR)
     split = 2 * R * H * 128 * dk * 2
+    units = R * 4 + (R + 1) * 4 + R * B * 96 * 4 + R * B * 16 + 16
     assert ola.ola_workspace_bytes(gt) == (expect + split + 2 * R * B * 4 + 2 * R * B * 4 +
-                                           R * B * T * 4)
+                                           units)
+    # tensor path, d_v = 64: the parent-chain table
+    dv2 = 64
+    g2 = _geom(R=2, H=3, d_k=64, d_v=dv2, B=40, T_max=5, in_dtype=ola.OLA_BF16,
+               math=ola.OLA_MATH_TENSOR)
+    expect2 = (R * H * dv2 * dk * 4 + T * R * H * B * dv2 * 4 + T * R * H * B * dk * 2 +
+               T * R * H * B * 4 + T * R * B * T * 4 + 16)
+    assert ola.ola_workspace_bytes(g2) == (expect2 + 2 * R * H * 128 * dk * 2 + 2 * R * B * 4 +
+                                           2 * R * B * 4 + R * B * T * 4)
 
 
 def test_null_arguments(L):

@@ -111,6 +111,25 @@ def test_max_steps_32():
     _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
 
 
+@pytest.mark.parametrize("d_k", [64, 128])
+def test_deep_chains_tensor_units(d_k):
+    """d_v = 128, chains of up to 11 records (T = 12, the deepest the tensor-core replay
+    accumulation takes) under steep Zipf pruning with a fan-out cap: units are cut at 48
+    distinct records, several per request."""
+    w = wl.WORKLOADS["stress"].scaled(R=2, H=2, d_k=d_k, B=300, P=64, T=12)
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_tensor"], S32, steps, dev_steps, parents)
+
+
+@pytest.mark.parametrize("B", [1024, 1025])
+def test_beam_count_limit_of_tensor_units(B):
+    """B = 1024 is the widest beam the unit-planned tensor kernel takes; 1025 goes to the
+    per-chunk kernel. Both must agree with the oracle."""
+    w = wl.WORKLOADS["single_request"].scaled(H=1, B=B, P=16, T=3)
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_tensor"], S32, steps, dev_steps, parents)
+
+
 def test_bf16_inputs_small_widths_fp32_path():
     w = wl.WORKLOADS["tiny"].scaled(dtype="bf16", d_k=32, d_v=16, B=12)
     S32, steps, dev_steps, parents = small_problem(w)
