@@ -22,15 +22,18 @@
 //
 // One CTA per SM walks the units of its (request, head) pairs, dealt round-robin, through a
 // three-stage ring. Warp roles:
-//   warps 0-1   producers: cp.async of the unit's q, k rows (128-byte swizzled K-major operand),
-//               distinct ancestor keys (swizzled) and w rows (MN-major operand); bulk copies
-//               of the v rows.
-//   warp 2      MMA: G with the staged q, k tile as A and the ancestor keys as B; D1 with S_ctx
-//               (bf16 hi + lo) held in tensor memory as the A operand; then D2 with the staged w
-//               planes as the A operand and Cf as B, written over G. Two accumulator stages.
-//   warps 3-6   builders: S_ctx into tensor memory when the (request, head) changes; per unit
-//               the decay table, k_p . q_p, Cf from G, and the appends of k_p and alpha_p.
-//   warps 7-14  epilogue: thread = state row i; w_p[i] and o_p[i] from D1, D2 and the scalars;
+//   warps 0-5   producers: TMA row gathers (tile::gather4, 128-byte swizzle) of the unit's q, k
+//               and v rows, distinct ancestor keys and w records (the latter as the MN-major
+//               operand), one list of copies dealt out in six chunks; cp.async of the
+//               per-position scalars.
+//   warp 6      MMA: G with the staged q, k tile as A and the ancestor keys as B; D1 with S_ctx
+//               (bf16 hi + lo) held in tensor memory as the A operand; D2 with the staged w
+//               planes as the A operand and Cf as B, written over G. Two accumulator stages;
+//               D2 of unit i - 1 is issued before G and D1 of unit i.
+//   warp 7      prep: decay table, k_p . q_p, per-position scalars, appends of k_p and alpha_p.
+//   warps 8-11  coefficients: S_ctx into tensor memory when the (request, head) changes; Cf
+//               from G and the decay table.
+//   warps 12-19 epilogue: thread = state row i; w_p[i] and o_p[i] from D1, D2 and the scalars;
 //               stores o (fp32) and the w record (hi, lo).
 // Every wait is bounded; on timeout the kernel records OLA_ERR_TIMEOUT and finishes.
 #include "ola_device.cuh"
@@ -41,12 +44,16 @@ constexpr int kMmaStages = 3;
 constexpr int kMmaMaxT = 12;
 constexpr int kMmaMaxB = 1024;
 constexpr int kMmaDV = 128;
-constexpr int kMmaProd = 2, kMmaCoef = 4, kMmaEpi = 8;
-constexpr int kMmaWarps = kMmaProd + 2 + kMmaCoef + kMmaEpi;   // 16 warps, 4 per subpartition
-constexpr int kMmaWMma = kMmaProd;              // warp 2
-constexpr int kMmaWPrep = kMmaProd + 1;         // warp 3
-constexpr int kMmaWCoef = kMmaProd + 2;         // warps 4..7 (subpartitions 0..3)
-constexpr int kMmaWEpi = kMmaWCoef + kMmaCoef;  // warps 8..15
+// A TMA instruction holds its warp for several hundred cycles plus roughly eighty per active
+// lane, while the instructions of different warps proceed in parallel: the copies of a unit are
+// spread over six producer warps, one warp-wide gather instruction each.
+constexpr int kMmaProd = 6, kMmaCoef = 4, kMmaEpi = 8;
+constexpr int kMmaWarps = kMmaProd + 2 + kMmaCoef + kMmaEpi;   // 20 warps, 5 per subpartition
+constexpr int kMmaWMma = kMmaProd;              // warp 6
+constexpr int kMmaWPrep = kMmaProd + 1;         // warp 7
+constexpr int kMmaWCoef = kMmaProd + 2;         // warps 8..11 (subpartitions 0..3)
+constexpr int kMmaWEpi = kMmaWCoef + kMmaCoef;  // warps 12..19
+static_assert(kMmaWCoef % 4 == 0 && kMmaWEpi % 4 == 0, "tensor-memory lane quarters follow warp % 4");
 
 // Record row of (step slot, request r, beam b, head h) in this kernel's record storage, which
 // keeps the heads of a beam next to each other: [T_max][R][B][H] (the heads of one beam are
@@ -73,7 +80,7 @@ struct MmaScal {                 // per position
 //   stage s: X [NSL][64 rows: q of positions 0-31 | k of positions 0-31][128 B]  K-major, sw128
 //            KA [NSL][48 rows][128 B]       ancestor keys, same swizzle
 //            WH, WL [6 groups of 8 records][2 halves of d_v][8][128 B]  MN-major, sw128
-//            V [32][d_v] bf16, MmaInfo
+//            V [2 halves of d_v][32 positions][128 B]  sw128, MmaInfo
 //   then CH, CL [64 rows][128 B] (Cf hi, lo; K-major, sw128), DEC [2][32][48] fp32,
 //   SC [2][32], barriers.
 struct MmaLayout {
@@ -103,12 +110,11 @@ template <int DK>
 __global__ void __launch_bounds__(kMmaWarps * 32, 1)
 replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* __restrict__ S_lo,
                   StepArgs a, UnitPlan up, const __grid_constant__ CUtensorMap mq,
-                  const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mkr,
-                  const __grid_constant__ CUtensorMap mw) {
+                  const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
+                  const __grid_constant__ CUtensorMap mkr, const __grid_constant__ CUtensorMap mw) {
   constexpr int NS = kMmaStages, DV = kMmaDV, UC = kUnitAnc, NP = kUnitPos;
   constexpr int CR = DK / 8;       // 16-byte chunks of a key row
   constexpr int NSL = DK / 64;     // 64-column slices of a key row
-  constexpr int CPL = DK / 32;     // chunks per lane when 4 lanes share a row
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = align_smem_1024(smem_raw);
   const MmaLayout L = mma_layout(DK);
@@ -181,7 +187,6 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       const int* rec = up.urec + (size_t(r) * up.maxU + k) * kUnitRecInts;
       int x0 = __ldcg(rec + lane), x1 = __ldcg(rec + 32 + lane), x2 = __ldcg(rec + 64 + lane);
       int prev_rh = -1;
-      const unsigned char* vg = static_cast<const unsigned char*>(a.v);
       for (int i = 0; i < n_my; ++i) {
         const int s = i % NS, n = i / NS;
         if (i >= NS && !__all_sync(kFull, mbar_wait_bounded(&empty[s], (n - 1) & 1))) {
@@ -240,10 +245,14 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         const int row1 = rec_row_hm(a, anc1 >> 16, r, h, anc1 & 0xffff);
         unsigned char* st = stage(s);
         MmaInfo* inf = info(s);
-        // every operand row goes in by TMA: q / k rows and ancestor keys / w records by row
-        // gathers of four (tile::gather4, 128-byte swizzle), v rows by bulk copies; all counted
-        // as transaction bytes on full[s]. Rows past n_pos / U repeat row 0 (never read).
-        const int U4 = (U + 3) & ~3;
+        // Every operand row goes in by TMA row gathers of four (tile::gather4, 128-byte
+        // swizzle, 64 columns per copy), all counted as transaction bytes on full[s]: q, k rows
+        // of the position groups, v rows, the ancestor keys and the w records (hi, lo x two
+        // halves of d_v). The copies form one list; warp pw issues entries [pw C, pw C + C) in
+        // one instruction. Rows past n_pos / U repeat row 0 (never read).
+        const int U4 = (U + 3) & ~3, G4 = (n_pos + 3) >> 2;
+        const int nqk = 2 * G4 * NSL, nv = 2 * G4, nka = (U4 / 4) * NSL;
+        const int nops = nqk + nv + nka + U4;
         if (pw == 0) {
           if (lane == 0) {
             inf->r = r;
@@ -256,57 +265,58 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           }
           inf->beam[lane] = beam;
           __syncwarp();
-          if (lane == 0)
-            mbar_arrive_expect_tx(&full[s], uint32_t(2 * NP * DK * 2 + U4 * DK * 2 + U4 * 512 +
-                                                     n_pos * DV * 2));
+          if (lane == 0) mbar_arrive_expect_tx(&full[s], uint32_t(nops) * 512u);
           __syncwarp();
-          // q, k rows: op = (side, group of four positions, 64-column slice)
-          {
-            const int id = lane;
-            const int side = id / (8 * NSL), m = (id / NSL) % 8, ks = id % NSL;
-            int y[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int pj = 4 * m + j;
-              y[j] = __shfl_sync(kFull, io_l, pj < n_pos ? pj : 0);
-            }
-            if (id < 16 * NSL)
-              tma_gather4(st + ks * 8192 + (side * NP + 4 * m) * 128, side ? &mk : &mq, &full[s],
-                          64 * ks, y[0], y[1], y[2], y[3]);
+        }
+        {
+          const int C = (nops + kMmaProd - 1) / kMmaProd;          // <= 20 (<= 120 copies)
+          const int id = pw * C + lane;
+          const bool has = lane < C && id < nops;
+          const int kind = id < nqk ? 0 : id < nqk + nv ? 1 : id < nqk + nv + nka ? 2 : 3;
+          int m, xc, sm_off;
+          const CUtensorMap* map;
+          if (kind == 0) {
+            const int side = id / (G4 * NSL), e = id % (G4 * NSL), ks = e % NSL;
+            m = e / NSL;
+            xc = 64 * ks;
+            sm_off = ks * 8192 + (side * NP + 4 * m) * 128;
+            map = side ? &mk : &mq;
+          } else if (kind == 1) {
+            const int e = id - nqk, ks = e & 1;
+            m = e >> 1;
+            xc = 64 * ks;
+            sm_off = int(L.v_off) + ks * (NP * 128) + 4 * m * 128;
+            map = &mv;
+          } else if (kind == 2) {
+            const int e = id - nqk - nv, ks = e % NSL;
+            m = e / NSL;
+            xc = 64 * ks;
+            sm_off = int(L.ka_off) + ks * (UC * 128) + 4 * m * 128;
+            map = &mkr;
+          } else {
+            const int e = id - nqk - nv - nka, pl = (e >> 1) & 1, mb = e & 1;
+            m = e >> 2;
+            xc = 128 * pl + 64 * mb;
+            sm_off = int(pl ? L.wl_off : L.wh_off) + (4 * m >> 3) * 2048 + mb * 1024 + (4 * m & 7) * 128;
+            map = &mw;
           }
-          if (lane < n_pos)
-            bulk_load(st + L.v_off + lane * (DV * 2), vg + size_t(io_l) * DV * 2, DV * 2, &full[s]);
+          int y[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int pj = (4 * m + j) & 63;
+            const int yp = __shfl_sync(kFull, io_l, pj < n_pos ? pj : 0);
+            const int uu = pj < U ? pj : 0;
+            const int rA = __shfl_sync(kFull, row0, uu & 31), rB = __shfl_sync(kFull, row1, uu & 31);
+            y[j] = kind <= 1 ? yp : (uu < 32 ? rA : rB);
+          }
+          if (has) tma_gather4(st + sm_off, map, &full[s], xc, y[0], y[1], y[2], y[3]);
+        }
+        if (pw == 1) {
           if (lane < n_pos) {
             cp_async4(&inf->gb[2 * lane], a.g + io_l);
             cp_async4(&inf->gb[2 * lane + 1], a.beta + io_l);
-          }
-        } else {
-          // ancestor keys (U4/4 x NSL gathers) then w records (U4/4 x 4: hi, lo x two halves)
-          const int nka = (U4 / 4) * NSL, nops = nka + U4;
-          for (int r0 = 0; r0 < nops; r0 += 32) {
-            const int id = r0 + lane;
-            const int m = id < nka ? id / NSL : (id - nka) >> 2;
-            int y[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int u = 4 * m + j;
-              const int uu = u < U ? u : 0;
-              const int rA = __shfl_sync(kFull, row0, uu & 31), rB = __shfl_sync(kFull, row1, uu & 31);
-              y[j] = uu < 32 ? rA : rB;
-            }
-            if (id < nka) {
-              const int ks = id % NSL;
-              tma_gather4(st + L.ka_off + ks * (UC * 128) + 4 * m * 128, &mkr, &full[s], 64 * ks,
-                          y[0], y[1], y[2], y[3]);
-            } else if (id < nops) {
-              const int pl = ((id - nka) >> 1) & 1, mb = (id - nka) & 1;
-              tma_gather4(st + (pl ? L.wl_off : L.wh_off) + (4 * m >> 3) * 2048 + mb * 1024 +
-                              (4 * m & 7) * 128,
-                          &mw, &full[s], 128 * pl + 64 * mb, y[0], y[1], y[2], y[3]);
-            }
-          }
-          if (lane < n_pos)
             cp_async16(&inf->upos[lane][0], up.upos + (size_t(r) * a.B + start + lane) * 16);
+          }
           if (lane < U) cp_async4(&inf->alpha[lane], a.A + row0);
           if (lane + 32 < U) cp_async4(&inf->alpha[32 + lane], a.A + row1);
         }
@@ -325,79 +335,88 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     for (int i = issued > NS ? issued - NS : 0; i < issued; ++i)
       mbar_wait_bounded(&full[i % NS], (i / NS) & 1);
   } else if (warp == kMmaWMma) {
-    // ------------------------------------------------------------------ MMA (lane 0)
+    // ------------------------------------------------------------------ MMA (whole warp)
+    // The warp runs converged; one elected lane issues each tensor-core instruction.
+    // Software-pipelined by one unit: iteration i first finishes unit i - 1 (D2 once its Cf is
+    // written, then the commits that hand it to the epilogue), then starts unit i (G, D1). The
+    // coefficient warps build Cf of unit i while the tensor pipe runs unit i's D1 and the
+    // epilogue drains unit i - 1.
     int sver = -1, last_i = -1;
+    int pU = 0, ps = 0, pac = 0, pj = 0, plast = 0;    // the unit whose D2 is pending
     bool ok = true;
-    for (int i = 0; i < n_my && ok; ++i) {
-      const int s = i % NS, n = i / NS, ac = i & 1;
-      if (lane == 0) {
-        ok = mbar_wait_bounded(&full[s], n & 1);
-        fence_proxy_async_smem();                    // cp.async data -> tensor-core reads
+    for (int i = 0; i <= n_my && ok; ++i) {
+      if (i >= 1) {
+        ok = __all_sync(kFull, mbar_wait_bounded(coef_ready, (i - 1) & 1));
+        tc_fence_after();
+        if (ok) {
+          const uint32_t d2 = tmem + uint32_t(pac) * 128u + 64u;
+          const uint32_t st = smem_u32(stage(ps));
+          const uint32_t id2 = idesc_bf16_f32_amn(128, 2 * NP);
+#pragma unroll 1
+          for (int kq = 0; kq < (pU + 15) / 16; ++kq) {
+            const uint64_t ah = sw128_mnmajor_desc(st + L.wh_off + kq * 4096, 1024, 2048);
+            const uint64_t al = sw128_mnmajor_desc(st + L.wl_off + kq * 4096, 1024, 2048);
+            const uint64_t bh = sw128_kmajor_desc(smem_u32(CH) + kq * 32);
+            const uint64_t bl = sw128_kmajor_desc(smem_u32(CL) + kq * 32);
+            umma_bf16_w(d2, ah, bh, id2, kq != 0 ? 1u : 0u);
+            umma_bf16_w(d2, al, bh, id2, 1u);
+            umma_bf16_w(d2, ah, bl, id2, 1u);
+          }
+          umma_commit_w(&acc_full[pac]);
+          umma_commit_w(coef_free);
+          umma_commit_w(&empty[ps]);
+          if (plast) umma_commit_w(&sfree[pj]);
+          last_i = i - 1;
+        }
+      }
+      if (ok && i < n_my) {
+        const int s = i % NS, n = i / NS, ac = i & 1;
+        ok = __all_sync(kFull, mbar_wait_bounded(&full[s], n & 1));
+        fence_proxy_async_smem();                  // cp.async data -> tensor-core reads
         const MmaInfo* inf = info(s);
         const int U = min(inf->U, UC);
-        const bool lastf = inf->last != 0;
         if (inf->first) ++sver;
         const int j = sver & 1;
-        if (i >= 2) ok = ok && mbar_wait_bounded(&acc_empty[ac], ((i - 2) >> 1) & 1);
+        if (i >= 2) ok = ok && __all_sync(kFull, mbar_wait_bounded(&acc_empty[ac], ((i - 2) >> 1) & 1));
         tc_fence_after();
         const uint32_t d1 = tmem + uint32_t(ac) * 128u, d2 = d1 + 64u;
-        const unsigned char* st = stage(s);
+        const uint32_t st = smem_u32(stage(s));
         if (ok && U > 0) {
-          // G[x][u] = x . k_u (M = 64 rows x of the q | k tile, N = 48 records), into the columns
-          // that D2 overwrites once the builders have read G
+          // G[x][u] = x . k_u (M = 64 rows x of the q | k tile, N = 48 records), into the
+          // columns that D2 overwrites once the coefficient warps have read G
           const uint32_t id0 = idesc_bf16_f32(64, UC);
-#pragma unroll
-          for (int ks = 0; ks < DK / 64; ++ks) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ax = sw128_kmajor_desc(smem_u32(st + ks * 8192) + kk * 32);
-              const uint64_t bk = sw128_kmajor_desc(smem_u32(st + L.ka_off + ks * (UC * 128)) + kk * 32);
-              umma_bf16(d2, ax, bk, id0, (ks | kk) != 0 ? 1u : 0u);
-            }
+#pragma unroll 1
+          for (int kstep = 0; kstep < DK / 16; ++kstep) {
+            const uint32_t ks = uint32_t(kstep >> 2), kk = uint32_t(kstep & 3);
+            const uint64_t ax = sw128_kmajor_desc(st + ks * 8192u + kk * 32u);
+            const uint64_t bk = sw128_kmajor_desc(st + L.ka_off + ks * (UC * 128u) + kk * 32u);
+            umma_bf16_w(d2, ax, bk, id0, kstep != 0 ? 1u : 0u);
           }
-          umma_commit(g_ready);
+          umma_commit_w(g_ready);
         }
-        ok = ok && mbar_wait_bounded(&sready[j], (sver >> 1) & 1);
+        ok = ok && __all_sync(kFull, mbar_wait_bounded(&sready[j], (sver >> 1) & 1));
         tc_fence_after();
         if (ok) {
           const uint32_t sa = tmem + 256u + uint32_t(j) * 128u;
           const uint32_t id1 = idesc_bf16_f32(128, 2 * NP);
-#pragma unroll
-          for (int ks = 0; ks < DK / 64; ++ks) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const int kstep = ks * 4 + kk;
-              const uint64_t bx = sw128_kmajor_desc(smem_u32(st + ks * 8192) + kk * 32);
-              umma_bf16_ts(d1, sa + kstep * 8, bx, id1, kstep != 0 ? 1u : 0u);
-              umma_bf16_ts(d1, sa + DK / 2 + kstep * 8, bx, id1, 1u);
-            }
+#pragma unroll 1
+          for (int kstep = 0; kstep < DK / 16; ++kstep) {
+            const uint32_t ks = uint32_t(kstep >> 2), kk = uint32_t(kstep & 3);
+            const uint64_t bx = sw128_kmajor_desc(st + ks * 8192u + kk * 32u);
+            umma_bf16_ts_w(d1, sa + kstep * 8, bx, id1, kstep != 0 ? 1u : 0u);
+            umma_bf16_ts_w(d1, sa + DK / 2 + kstep * 8, bx, id1, 1u);
           }
-          ok = mbar_wait_bounded(coef_ready, i & 1);
-          tc_fence_after();
-          if (ok && U > 0) {
-            const uint32_t id2 = idesc_bf16_f32_amn(128, 2 * NP);
-            for (int kq = 0; kq < (U + 15) / 16; ++kq) {
-              const uint64_t ah = sw128_mnmajor_desc(smem_u32(st + L.wh_off) + kq * 4096, 1024, 2048);
-              const uint64_t al = sw128_mnmajor_desc(smem_u32(st + L.wl_off) + kq * 4096, 1024, 2048);
-              const uint64_t bh = sw128_kmajor_desc(smem_u32(CH) + kq * 32);
-              const uint64_t bl = sw128_kmajor_desc(smem_u32(CL) + kq * 32);
-              umma_bf16(d2, ah, bh, id2, kq != 0 ? 1u : 0u);
-              umma_bf16(d2, al, bh, id2, 1u);
-              umma_bf16(d2, ah, bl, id2, 1u);
-            }
-          }
-          umma_commit(&acc_full[ac]);
-          umma_commit(coef_free);
-          umma_commit(&empty[s]);
-          if (lastf) umma_commit(&sfree[j]);
-          last_i = i;
         }
-        if (!ok) report_error(a.err, OLA_ERR_TIMEOUT, 21, t);
+        pU = U;
+        ps = s;
+        pac = ac;
+        pj = j;
+        plast = inf->last;
       }
-      ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+      if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 21, t);
     }
     // tensor memory is released only once the last MMA has completed
-    if (lane == 0 && last_i >= 0) mbar_wait_bounded(&acc_full[last_i & 1], (last_i >> 1) & 1);
+    if (last_i >= 0) mbar_wait_bounded(&acc_full[last_i & 1], (last_i >> 1) & 1);
     __syncwarp();
   } else if (warp == kMmaWPrep) {
     // ------------------------------------------------------------------ prep warp
@@ -470,7 +489,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         for (int m = 0; m < 2; ++m)
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) acc[m][hh][0] = acc[m][hh][1] = acc[m][hh][2] = acc[m][hh][3] = 0.f;
-#pragma unroll
+#pragma unroll 2
         for (int kq = 0; kq < DK / 16; ++kq) {
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
@@ -497,7 +516,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       {
         constexpr int RPI = 32 / CR;
         const int c = lane % CR;
-#pragma unroll
+#pragma unroll 4
         for (int j = 0; j < NP / RPI; ++j) {
           const int pp = j * RPI + lane / CR, nn = 32 + pp;
           const int wr = __shfl_sync(kFull, wnew, pp);
@@ -533,8 +552,8 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           break;
         }
         // S_ctx rows 32 sp .. 32 sp + 31 (hi, then lo) into buffer j; one row per lane, two bf16
-        // per 32-bit column, lower k in the low half (memory order); eight 16-byte loads at a
-        // time (the rows were prefetched into L2 by the producers)
+        // per 32-bit column, lower k in the low half (memory order); four 16-byte loads per
+        // tensor-memory store (the rows were prefetched into L2 by the producers)
         tc_fence_after();
         const int row = 32 * sp + lane;
         const size_t rh = size_t(r) * a.H + h;
@@ -543,16 +562,11 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         for (int half = 0; half < 2; ++half) {
           const uint4* src = reinterpret_cast<const uint4*>((half ? S_lo : S_hi) +
                                                             (rh * DV + row) * DK);
-#pragma unroll
-          for (int c8 = 0; c8 < DK / 64; ++c8) {
-            uint4 v[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) v[c] = __ldg(src + 8 * c8 + c);
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const uint4 w4[4] = {v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]};
-              tmem_st16(ta + half * (DK / 2) + (2 * c8 + c) * 16, w4);
-            }
+#pragma unroll 1
+          for (int c4 = 0; c4 < DK / 32; ++c4) {
+            const uint4 w4[4] = {__ldg(src + 4 * c4), __ldg(src + 4 * c4 + 1), __ldg(src + 4 * c4 + 2),
+                                 __ldg(src + 4 * c4 + 3)};
+            tmem_st16(ta + half * (DK / 2) + c4 * 16, w4);
           }
         }
         tmem_st_wait();
@@ -581,7 +595,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         const uint32_t tg = tmem + (uint32_t(32 * sp) << 16) + uint32_t(ac) * 128u + 64u;
         const int nrow = 16 * sp + (lane & 15), p = nrow & 31;
         const float* dr = DEC0 + ac * (NP * UC) + p * UC;
-#pragma unroll
+#pragma unroll 1
         for (int h16 = 0; h16 < UC / 16; ++h16) {
           if (16 * h16 >= U) break;                   // warp-uniform
           float gr[16];
@@ -638,11 +652,11 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       }
       tc_fence_after();
       const MmaScal* sc = SC + ac * NP;
-      const __nv_bfloat16* Vs = reinterpret_cast<const __nv_bfloat16*>(stage(s) + L.v_off);
+      const unsigned char* Vb = stage(s) + L.v_off;   // [2][32][128 B] sw128
       const MmaInfo* inf = info(s);
       const int n_pos = min(inf->n_pos, NP), U = inf->U;
       const uint32_t base = tl + uint32_t(ac) * 128u;
-#pragma unroll
+#pragma unroll 1
       for (int pb = 0; pb < 2; ++pb) {
         const int p0 = 16 * ph + 8 * pb;
         if (p0 < n_pos) {                             // warp-uniform
@@ -653,20 +667,38 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
 #pragma unroll
             for (int j = 0; j < 8; ++j) q2[j] = k2[j] = 0.f;
           }
+          // four positions at a time: their scalars and v first, then the stores (loads issued
+          // ahead of the stores, which the compiler cannot move them past)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const MmaScal e = sc[p0 + j];
-            if (e.valid) {
-              const float uu = fmaf(e.e, k1[j], k2[j]);
-              const float qq = fmaf(e.e, q1[j], q2[j]);
-              const float v = __bfloat162float(Vs[(p0 + j) * DV + row]);
-              const float w = e.beta * (v - e.alpha * uu);
-              const float o = fmaf(e.alpha, qq, e.c0 * w);
-              a.o[size_t(e.io) * DV + row] = o;
-              const __nv_bfloat16 whi = __float2bfloat16_rn(w);
-              const __nv_bfloat16 wlo = __float2bfloat16_rn(w - __bfloat162float(whi));
-              Wb[size_t(e.wnew) * (2 * DV) + row] = whi;
-              Wb[size_t(e.wnew) * (2 * DV) + DV + row] = wlo;
+          for (int j4 = 0; j4 < 8; j4 += 4) {
+            float4 sa[4];
+            int io[4], wn[4];
+            float vv[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const int pp = p0 + j4 + jj;
+              sa[jj] = *reinterpret_cast<const float4*>(&sc[pp]);
+              const int4 sb = *reinterpret_cast<const int4*>(&sc[pp].io);
+              io[jj] = sb.x;
+              wn[jj] = sb.y;
+              vv[jj] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                  Vb + (row >> 6) * (NP * 128) + pp * 128 + ((((row & 63) >> 3) ^ (pp & 7)) << 4) +
+                  (row & 7) * 2));
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const int j = j4 + jj;
+              if (p0 + j < n_pos) {
+                const float uu = fmaf(sa[jj].x, k1[j], k2[j]);
+                const float qq = fmaf(sa[jj].x, q1[j], q2[j]);
+                const float w = sa[jj].z * (vv[jj] - sa[jj].y * uu);
+                const float o = fmaf(sa[jj].y, qq, sa[jj].w * w);
+                a.o[size_t(io[jj]) * DV + row] = o;
+                const __nv_bfloat16 whi = __float2bfloat16_rn(w);
+                const __nv_bfloat16 wlo = __float2bfloat16_rn(w - __bfloat162float(whi));
+                Wb[size_t(wn[jj]) * (2 * DV) + row] = whi;
+                Wb[size_t(wn[jj]) * (2 * DV) + DV + row] = wlo;
+              }
             }
           }
         }
@@ -711,7 +743,8 @@ bool make_record_maps(CUtensorMap* mkr, CUtensorMap* mw, const void* Kr, const v
 template <int DK>
 static cudaError_t launch_mma_t(const void* S_hi, const void* S_lo, const StepArgs& a,
                                 const UnitPlan& up, const CUtensorMap& mq, const CUtensorMap& mk,
-                                const CUtensorMap& mkr, const CUtensorMap& mw, int n_sm,
+                                const CUtensorMap& mv, const CUtensorMap& mkr, const CUtensorMap& mw,
+                                int n_sm,
                                 cudaStream_t stream) {
   const MmaLayout L = mma_layout(DK);
   auto kern = replay_mma_kernel<DK>;
@@ -720,20 +753,21 @@ static cudaError_t launch_mma_t(const void* S_hi, const void* S_lo, const StepAr
   if (e != cudaSuccess) return e;
   kern<<<n_sm, kMmaWarps * 32, L.bytes, stream>>>(static_cast<const __nv_bfloat16*>(S_hi),
                                                   static_cast<const __nv_bfloat16*>(S_lo), a, up,
-                                                  mq, mk, mkr, mw);
+                                                  mq, mk, mv, mkr, mw);
   return cudaGetLastError();
 }
 
 // S_hi, S_lo: the shared state split into bf16 hi + lo, [R*H][128][d_k]. W records are stored
 // as [hi plane | lo plane] bf16 rows of 2 d_v elements. mkr, mw from make_record_maps; the
-// q and k maps are made here for this step's inputs.
+// q, k and v maps are made here for this step's inputs.
 cudaError_t launch_replay_mma(const StepArgs& a, const UnitPlan& up, const void* S_hi,
                               const void* S_lo, const CUtensorMap& mkr, const CUtensorMap& mw,
                               cudaStream_t stream) {
-  CUtensorMap mq, mk;
+  CUtensorMap mq, mk, mv;
   const uint64_t rows = uint64_t(a.R) * a.B * a.H;
   if (!make_rows_map(&mq, a.q, rows, a.d_k, uint64_t(a.d_k) * 2) ||
-      !make_rows_map(&mk, a.k, rows, a.d_k, uint64_t(a.d_k) * 2))
+      !make_rows_map(&mk, a.k, rows, a.d_k, uint64_t(a.d_k) * 2) ||
+      !make_rows_map(&mv, a.v, rows, kMmaDV, uint64_t(kMmaDV) * 2))
     return cudaErrorInvalidValue;
   cudaError_t e = launch_plan_units(a, up, stream);
   if (e != cudaSuccess) return e;
@@ -741,8 +775,8 @@ cudaError_t launch_replay_mma(const StepArgs& a, const UnitPlan& up, const void*
   e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  if (a.d_k == 64) return launch_mma_t<64>(S_hi, S_lo, a, up, mq, mk, mkr, mw, n_sm, stream);
-  if (a.d_k == 128) return launch_mma_t<128>(S_hi, S_lo, a, up, mq, mk, mkr, mw, n_sm, stream);
+  if (a.d_k == 64) return launch_mma_t<64>(S_hi, S_lo, a, up, mq, mk, mv, mkr, mw, n_sm, stream);
+  if (a.d_k == 128) return launch_mma_t<128>(S_hi, S_lo, a, up, mq, mk, mv, mkr, mw, n_sm, stream);
   return cudaErrorInvalidValue;
 }
 
