@@ -22,38 +22,44 @@
 //
 // One CTA per SM walks the units of its (request, head) pairs, dealt round-robin, through a
 // three-stage ring. Warp roles:
-//   warps 0-5   producers: TMA row gathers (tile::gather4, 128-byte swizzle) of the unit's q, k
-//               and v rows, distinct ancestor keys and w records (the latter as the MN-major
-//               operand), one list of copies dealt out in six chunks; cp.async of the
+//   warps 0-2, 4-6  producers: TMA row gathers (tile::gather4, 128-byte swizzle) of the unit's
+//               q, k and v rows, distinct ancestor keys and w records (the latter as the
+//               MN-major operand), one list of copies dealt out in six chunks; cp.async of the
 //               per-position scalars.
-//   warp 6      MMA: G with the staged q, k tile as A and the ancestor keys as B; D1 with S_ctx
+//   warp 3      MMA: G with the staged q, k tile as A and the ancestor keys as B; D1 with S_ctx
 //               (bf16 hi + lo) held in tensor memory as the A operand; D2 with the staged w
-//               planes as the A operand and Cf as B, written over G. Two accumulator stages;
+//               planes as the A operand and Cf as B, written over G. Three accumulator stages;
 //               D2 of unit i - 1 is issued before G and D1 of unit i.
-//   warp 7      prep: decay table, k_p . q_p, per-position scalars, appends of k_p and alpha_p.
-//   warps 8-11  coefficients: S_ctx into tensor memory when the (request, head) changes; Cf
-//               from G and the decay table.
+//   warp 7      prep: decay table, per-position scalars, append of alpha_p.
+//   warps 8-11  coefficients: S_ctx into tensor memory when the (request, head) changes;
+//               k_p . q_p; Cf from G and the decay table.
 //   warps 12-19 epilogue: thread = state row i; w_p[i] and o_p[i] from D1, D2 and the scalars;
-//               stores o (fp32) and the w record (hi, lo).
+//               stores o (fp32), the w record (hi, lo) and the k_p record.
 // Every wait is bounded; on timeout the kernel records OLA_ERR_TIMEOUT and finishes.
 #include "ola_device.cuh"
 
 namespace ola {
 
-constexpr int kMmaStages = 3;
+constexpr int kMmaStages = 3;    // operand stages in shared memory
+constexpr int kMmaAcc = 3;       // accumulator stages in tensor memory (and scalar / decay buffers)
 constexpr int kMmaMaxT = 12;
 constexpr int kMmaMaxB = 1024;
 constexpr int kMmaDV = 128;
 // A TMA instruction holds its warp for several hundred cycles plus roughly eighty per active
 // lane, while the instructions of different warps proceed in parallel: the copies of a unit are
 // spread over six producer warps, one warp-wide gather instruction each.
+// Warp w runs on subpartition w % 4. Every subpartition holds one coefficient warp and two
+// epilogue warps (their tensor-memory lane quarter is w % 4); the producers fill subpartitions
+// 0-2 and the MMA and prep warps share subpartition 3, so that each subpartition's warps run
+// few distinct loops (the instruction cache is small next to this kernel).
 constexpr int kMmaProd = 6, kMmaCoef = 4, kMmaEpi = 8;
 constexpr int kMmaWarps = kMmaProd + 2 + kMmaCoef + kMmaEpi;   // 20 warps, 5 per subpartition
-constexpr int kMmaWMma = kMmaProd;              // warp 6
-constexpr int kMmaWPrep = kMmaProd + 1;         // warp 7
-constexpr int kMmaWCoef = kMmaProd + 2;         // warps 8..11 (subpartitions 0..3)
+constexpr int kMmaWMma = 3;                     // subpartition 3
+constexpr int kMmaWPrep = 7;                    // subpartition 3
+constexpr int kMmaWCoef = 8;                    // warps 8..11 (subpartitions 0..3)
 constexpr int kMmaWEpi = kMmaWCoef + kMmaCoef;  // warps 12..19
 static_assert(kMmaWCoef % 4 == 0 && kMmaWEpi % 4 == 0, "tensor-memory lane quarters follow warp % 4");
+static_assert(kMmaWCoef == kMmaProd + 2, "warps 0..7 are the producers, the MMA and the prep warp");
 
 // Record row of (step slot, request r, beam b, head h) in this kernel's record storage, which
 // keeps the heads of a beam next to each other: [T_max][R][B][H] (the heads of one beam are
@@ -81,8 +87,8 @@ struct MmaScal {                 // per position
 //            KA [NSL][48 rows][128 B]       ancestor keys, same swizzle
 //            WH, WL [6 groups of 8 records][2 halves of d_v][8][128 B]  MN-major, sw128
 //            V [2 halves of d_v][32 positions][128 B]  sw128, MmaInfo
-//   then CH, CL [64 rows][128 B] (Cf hi, lo; K-major, sw128), DEC [2][32][48] fp32,
-//   SC [2][32], barriers.
+//   then CH, CL [64 rows][128 B] (Cf hi, lo; K-major, sw128), DEC [3][32][48] fp32,
+//   SC [3][32], barriers.
 struct MmaLayout {
   uint32_t ka_off, wh_off, wl_off, v_off, info_off, stage;
   uint32_t ch_off, cl_off, dec_off, sc_off, bar_off, bytes;
@@ -100,8 +106,8 @@ __host__ __device__ inline MmaLayout mma_layout(int d_k) {
   L.ch_off = uint32_t(kMmaStages) * L.stage;
   L.cl_off = L.ch_off + 8192u;
   L.dec_off = L.cl_off + 8192u;
-  L.sc_off = L.dec_off + 2u * kUnitPos * kUnitAnc * 4u;
-  L.bar_off = L.sc_off + 2u * kUnitPos * uint32_t(sizeof(MmaScal));
+  L.sc_off = L.dec_off + uint32_t(kMmaAcc) * kUnitPos * kUnitAnc * 4u;
+  L.bar_off = L.sc_off + uint32_t(kMmaAcc) * kUnitPos * uint32_t(sizeof(MmaScal));
   L.bytes = L.bar_off + 256u + 1024u;
   return L;
 }
@@ -112,31 +118,32 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
                   StepArgs a, UnitPlan up, const __grid_constant__ CUtensorMap mq,
                   const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                   const __grid_constant__ CUtensorMap mkr, const __grid_constant__ CUtensorMap mw) {
-  constexpr int NS = kMmaStages, DV = kMmaDV, UC = kUnitAnc, NP = kUnitPos;
+  constexpr int NS = kMmaStages, NA = kMmaAcc, DV = kMmaDV, UC = kUnitAnc, NP = kUnitPos;
   constexpr int CR = DK / 8;       // 16-byte chunks of a key row
   constexpr int NSL = DK / 64;     // 64-column slices of a key row
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = align_smem_1024(smem_raw);
   const MmaLayout L = mma_layout(DK);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* full = bars;             // [NS] stage loaded: cp.async arrivals + 1, TMA bytes
-  uint64_t* empty = bars + 3;        // [NS] stage consumed: MMA commit, prep warp, epilogue warps
-  uint64_t* acc_full = bars + 6;     // [2] accumulators of a unit complete
-  uint64_t* acc_empty = bars + 8;    // [2] epilogue done with an accumulator stage
-  uint64_t* scal_ready = bars + 10;  // [2] per-position scalars written
-  uint64_t* coef_ready = bars + 12;  // Cf of the current unit written (every unit)
-  uint64_t* coef_free = bars + 13;   // MMAs of the previous unit done (Cf may be rewritten)
-  uint64_t* sready = bars + 14;      // [2] S_ctx buffer loaded into tensor memory
-  uint64_t* sfree = bars + 16;       // [2] last MMA reading an S_ctx buffer done
-  uint64_t* dec_ready = bars + 18;   // [2] decay table buffer written
-  uint64_t* dec_free = bars + 20;    // [2] coefficient warps done with a decay table buffer
-  uint64_t* g_ready = bars + 22;     // G of the current unit in tensor memory (units with U > 0)
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 23);
+  uint64_t* full = bars;               // [NS] stage loaded: cp.async arrivals + 1, TMA bytes
+  uint64_t* empty = full + NS;         // [NS] stage consumed: MMA commit, prep warp, epilogue warps
+  uint64_t* acc_full = empty + NS;     // [NA] accumulators of a unit complete
+  uint64_t* acc_empty = acc_full + NA; // [NA] epilogue done with an accumulator stage
+  uint64_t* scal_ready = acc_empty + NA;  // [NA] per-position scalars written
+  uint64_t* dec_ready = scal_ready + NA;  // [NA] decay table buffer written
+  uint64_t* dec_free = dec_ready + NA;    // [NA] coefficient warps done with a decay table buffer
+  uint64_t* coef_ready = dec_free + NA;   // Cf of the current unit written (every unit)
+  uint64_t* coef_free = coef_ready + 1;   // MMAs of the previous unit done (Cf may be rewritten)
+  uint64_t* sready = coef_free + 1;    // S_ctx loaded into tensor memory
+  uint64_t* sfree = sready + 1;        // last MMA reading S_ctx done
+  uint64_t* g_ready = sfree + 1;       // G of the current unit in tensor memory (units with U > 0)
+  uint32_t* holder = reinterpret_cast<uint32_t*>(g_ready + 1);
+  static_assert((2 * NS + 5 * NA + 5) * 8 + 8 <= 256, "barrier area");
   auto stage = [&](int s) { return smem + size_t(s) * L.stage; };
   auto info = [&](int s) { return reinterpret_cast<MmaInfo*>(stage(s) + L.info_off); };
   unsigned char* CH = smem + L.ch_off;
   unsigned char* CL = smem + L.cl_off;
-  float* DEC0 = reinterpret_cast<float*>(smem + L.dec_off);   // [2][32][48]
+  float* DEC0 = reinterpret_cast<float*>(smem + L.dec_off);   // [NA][32][48]
   MmaScal* SC = reinterpret_cast<MmaScal*>(smem + L.sc_off);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -152,17 +159,17 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       mbar_init(&full[s], 32 * kMmaProd + 1);   // cp.async arrivals + header (with bytes)
       mbar_init(&empty[s], 1 + 1 + kMmaEpi);
     }
-    for (int x = 0; x < 2; ++x) {
+    for (int x = 0; x < NA; ++x) {
       mbar_init(&acc_full[x], 1);
       mbar_init(&acc_empty[x], kMmaEpi);
-      mbar_init(&scal_ready[x], 1);
-      mbar_init(&sready[x], kMmaCoef);
-      mbar_init(&sfree[x], 1);
+      mbar_init(&scal_ready[x], 1 + kMmaCoef);   // prep warp, c0 from the coefficient warps
       mbar_init(&dec_ready[x], 1);
       mbar_init(&dec_free[x], kMmaCoef);
     }
     mbar_init(coef_ready, kMmaCoef);
     mbar_init(coef_free, 1);
+    mbar_init(sready, kMmaCoef);
+    mbar_init(sfree, 1);
     mbar_init(g_ready, 1);
     fence_barrier_init();
   }
@@ -173,16 +180,17 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
   fence_proxy_async_smem();
   __syncthreads();
   tc_fence_after();
-  // tensor memory: columns [128 a, 128 a + 128) accumulator stage a (D1 q | D1 k | D2 q | D2 k),
-  // [256 + 128 j, +128) S_ctx buffer j (hi in the first d_k / 2 columns, lo after)
+  // tensor memory: columns [128 a, 128 a + 128) accumulator stage a < 3 (D1 q | D1 k | D2 q |
+  // D2 k), [384, 512) S_ctx (hi in the first d_k / 2 columns, lo after)
   const uint32_t tmem = *holder;
 
-  if (warp < kMmaProd) {
+  if (warp < kMmaWCoef && warp != kMmaWMma && warp != kMmaWPrep) {
     // ------------------------------------------------------------------ producers
-    const int pw = warp;
+    const int pw = warp < kMmaWMma ? warp : warp - 1;     // 0..5
     int issued = 0;
     if (n_my > 0) {
       int r = int(blockIdx.x) / a.H, h = int(blockIdx.x) % a.H, k = 0;
+      const int dr = int(gridDim.x) / a.H, dh = int(gridDim.x) % a.H;   // the walk's stride
       int cnt = __ldcg(up.ucnt + r);
       const int* rec = up.urec + (size_t(r) * up.maxU + k) * kUnitRecInts;
       int x0 = __ldcg(rec + lane), x1 = __ldcg(rec + 32 + lane), x2 = __ldcg(rec + 64 + lane);
@@ -197,9 +205,12 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         int nr = r, nh = h, nk = k + 1, ncnt = cnt;
         if (nk == cnt) {
           nk = 0;
-          const int nrh = r * a.H + h + int(gridDim.x);
-          nr = nrh / a.H;
-          nh = nrh % a.H;
+          nr = r + dr;
+          nh = h + dh;
+          if (nh >= a.H) {
+            nh -= a.H;
+            ++nr;
+          }
         }
         const bool more = i + 1 < n_my;
         int y0 = 0, y1 = 0, y2 = 0;
@@ -276,7 +287,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           int m, xc, sm_off;
           const CUtensorMap* map;
           if (kind == 0) {
-            const int side = id / (G4 * NSL), e = id % (G4 * NSL), ks = e % NSL;
+            const int side = id >= G4 * NSL ? 1 : 0, e = id - side * G4 * NSL, ks = e % NSL;
             m = e / NSL;
             xc = 64 * ks;
             sm_off = ks * 8192 + (side * NP + 4 * m) * 128;
@@ -342,7 +353,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     // coefficient warps build Cf of unit i while the tensor pipe runs unit i's D1 and the
     // epilogue drains unit i - 1.
     int sver = -1, last_i = -1;
-    int pU = 0, ps = 0, pac = 0, pj = 0, plast = 0;    // the unit whose D2 is pending
+    int pU = 0, ps = 0, pac = 0, plast = 0;             // the unit whose D2 is pending
     bool ok = true;
     for (int i = 0; i <= n_my && ok; ++i) {
       if (i >= 1) {
@@ -365,19 +376,18 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           umma_commit_w(&acc_full[pac]);
           umma_commit_w(coef_free);
           umma_commit_w(&empty[ps]);
-          if (plast) umma_commit_w(&sfree[pj]);
+          if (plast) umma_commit_w(sfree);
           last_i = i - 1;
         }
       }
       if (ok && i < n_my) {
-        const int s = i % NS, n = i / NS, ac = i & 1;
+        const int s = i % NS, n = i / NS, ac = i % NA;
         ok = __all_sync(kFull, mbar_wait_bounded(&full[s], n & 1));
         fence_proxy_async_smem();                  // cp.async data -> tensor-core reads
         const MmaInfo* inf = info(s);
         const int U = min(inf->U, UC);
         if (inf->first) ++sver;
-        const int j = sver & 1;
-        if (i >= 2) ok = ok && __all_sync(kFull, mbar_wait_bounded(&acc_empty[ac], ((i - 2) >> 1) & 1));
+        if (i >= NA) ok = ok && __all_sync(kFull, mbar_wait_bounded(&acc_empty[ac], ((i - NA) / NA) & 1));
         tc_fence_after();
         const uint32_t d1 = tmem + uint32_t(ac) * 128u, d2 = d1 + 64u;
         const uint32_t st = smem_u32(stage(s));
@@ -394,10 +404,10 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           }
           umma_commit_w(g_ready);
         }
-        ok = ok && __all_sync(kFull, mbar_wait_bounded(&sready[j], (sver >> 1) & 1));
+        ok = ok && __all_sync(kFull, mbar_wait_bounded(sready, sver & 1));
         tc_fence_after();
         if (ok) {
-          const uint32_t sa = tmem + 256u + uint32_t(j) * 128u;
+          const uint32_t sa = tmem + 128u * NA;
           const uint32_t id1 = idesc_bf16_f32(128, 2 * NP);
 #pragma unroll 1
           for (int kstep = 0; kstep < DK / 16; ++kstep) {
@@ -410,27 +420,23 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         pU = U;
         ps = s;
         pac = ac;
-        pj = j;
         plast = inf->last;
       }
       if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 21, t);
     }
     // tensor memory is released only once the last MMA has completed
-    if (last_i >= 0) mbar_wait_bounded(&acc_full[last_i & 1], (last_i >> 1) & 1);
+    if (last_i >= 0) mbar_wait_bounded(&acc_full[last_i % NA], (last_i / NA) & 1);
     __syncwarp();
   } else if (warp == kMmaWPrep) {
     // ------------------------------------------------------------------ prep warp
     // Per unit, from the staged data only (nothing here waits for a tensor-core result, so the
-    // warp runs ahead): k_p . q_p, the appends of k_p and alpha_p, the decay table and the
-    // per-position scalars.
-    __nv_bfloat16* kout = static_cast<__nv_bfloat16*>(a.Kr);
-    const int gq = lane >> 2, c4 = lane & 3;
+    // warp runs ahead): the decay table, the per-position scalars and the append of alpha_p.
     for (int i = 0; i < n_my; ++i) {
-      const int s = i % NS, n = i / NS, ac = i & 1;
+      const int s = i % NS, n = i / NS, ac = i % NA;
       bool ok = mbar_wait_bounded(&full[s], n & 1);
-      if (i >= 2) {
-        ok = ok && mbar_wait_bounded(&acc_empty[ac], ((i - 2) >> 1) & 1);   // SC[ac] free
-        ok = ok && mbar_wait_bounded(&dec_free[ac], ((i - 2) >> 1) & 1);    // DEC[ac] free
+      if (i >= NA) {
+        ok = ok && mbar_wait_bounded(&acc_empty[ac], ((i - NA) / NA) & 1);   // SC[ac] free
+        ok = ok && mbar_wait_bounded(&dec_free[ac], ((i - NA) / NA) & 1);    // DEC[ac] free
       }
       if (!__all_sync(kFull, ok)) {
         if (lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 23, t);
@@ -481,52 +487,6 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       sc[p].io = (r * a.B + b) * a.H + h;
       sc[p].wnew = wnew;
       sc[p].valid = valid ? 1 : 0;
-      // k_p . q_p: the diagonal of Xq Xk^T on warp-level MMA, 16 x 8 tiles along the diagonal
-      {
-        const uint32_t xb = smem_u32(st);
-        float acc[2][2][4];
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) acc[m][hh][0] = acc[m][hh][1] = acc[m][hh][2] = acc[m][hh][3] = 0.f;
-#pragma unroll 2
-        for (int kq = 0; kq < DK / 16; ++kq) {
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const int an = 16 * m + (lane & 15), kc = 2 * kq + (lane >> 4);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(xb + (kc >> 3) * 8192 + an * 128 + (((kc & 7) ^ (an & 7)) << 4), a0, a1, a2, a3);
-            const int bn = 32 + 16 * m + 8 * (lane >> 4) + (lane & 7), bc = 2 * kq + ((lane >> 3) & 1);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(xb + (bc >> 3) * 8192 + bn * 128 + (((bc & 7) ^ (bn & 7)) << 4), b0, b1, b2, b3);
-            mma_16816_bf16(acc[m][0], a0, a1, a2, a3, b0, b1);
-            mma_16816_bf16(acc[m][1], a0, a1, a2, a3, b2, b3);
-          }
-        }
-        // lane (g, c) with c = g / 2 holds the diagonal entries of rows g and g + 8 of a tile
-        if (c4 == (gq >> 1)) {
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            sc[16 * m + gq].c0 = (gq & 1) ? acc[m][0][1] : acc[m][0][0];
-            sc[16 * m + 8 + gq].c0 = (gq & 1) ? acc[m][1][3] : acc[m][1][2];
-          }
-        }
-      }
-      // append k_p (two rows of 256 bytes per warp instruction)
-      {
-        constexpr int RPI = 32 / CR;
-        const int c = lane % CR;
-#pragma unroll 4
-        for (int j = 0; j < NP / RPI; ++j) {
-          const int pp = j * RPI + lane / CR, nn = 32 + pp;
-          const int wr = __shfl_sync(kFull, wnew, pp);
-          if (pp < n_pos) {
-            const uint4 v = *reinterpret_cast<const uint4*>(
-                st + (c >> 3) * 8192 + nn * 128 + (((c & 7) ^ (nn & 7)) << 4));
-            *reinterpret_cast<uint4*>(kout + size_t(wr) * DK + c * 8) = v;
-          }
-        }
-      }
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&dec_ready[ac]);
@@ -539,45 +499,72 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     const int sp = warp & 3;
     int sver = -1, gcnt = 0;
     for (int i = 0; i < n_my; ++i) {
-      const int s = i % NS, n = i / NS, ac = i & 1;
+      const int s = i % NS, n = i / NS, ac = i % NA;
       bool ok = mbar_wait_bounded(&full[s], n & 1);
       const MmaInfo* inf = info(s);
       const int r = inf->r, h = inf->h, U = min(inf->U, UC);
       if (inf->first) {
         ++sver;
-        const int j = sver & 1;
-        if (sver >= 2) ok = ok && mbar_wait_bounded(&sfree[j], ((sver >> 1) - 1) & 1);
+        if (sver >= 1) ok = ok && mbar_wait_bounded(sfree, (sver - 1) & 1);
         if (!__all_sync(kFull, ok)) {
           if (lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 22, t);
           break;
         }
-        // S_ctx rows 32 sp .. 32 sp + 31 (hi, then lo) into buffer j; one row per lane, two bf16
-        // per 32-bit column, lower k in the low half (memory order); four 16-byte loads per
-        // tensor-memory store (the rows were prefetched into L2 by the producers)
+        // S_ctx rows 32 sp .. 32 sp + 31 (hi, then lo) into tensor memory; one row per lane, two
+        // bf16 per 32-bit column, lower k in the low half (memory order); eight 16-byte loads in
+        // flight per thread (the rows were prefetched into L2 by the producers)
         tc_fence_after();
         const int row = 32 * sp + lane;
         const size_t rh = size_t(r) * a.H + h;
-        const uint32_t ta = tmem + (uint32_t(32 * sp) << 16) + 256u + uint32_t(j) * 128u;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint4* src = reinterpret_cast<const uint4*>((half ? S_lo : S_hi) +
-                                                            (rh * DV + row) * DK);
+        const uint32_t ta = tmem + (uint32_t(32 * sp) << 16) + 128u * NA;
 #pragma unroll 1
-          for (int c4 = 0; c4 < DK / 32; ++c4) {
-            const uint4 w4[4] = {__ldg(src + 4 * c4), __ldg(src + 4 * c4 + 1), __ldg(src + 4 * c4 + 2),
-                                 __ldg(src + 4 * c4 + 3)};
-            tmem_st16(ta + half * (DK / 2) + c4 * 16, w4);
-          }
+        for (int c8 = 0; c8 < DK / 32; ++c8) {          // DK / 64 batches per half
+          const int half = c8 / (DK / 64), cb = c8 % (DK / 64);
+          const uint4* src = reinterpret_cast<const uint4*>((half ? S_lo : S_hi) + (rh * DV + row) * DK) + 8 * cb;
+          const uint4 w0[4] = {__ldg(src), __ldg(src + 1), __ldg(src + 2), __ldg(src + 3)};
+          const uint4 w1[4] = {__ldg(src + 4), __ldg(src + 5), __ldg(src + 6), __ldg(src + 7)};
+          tmem_st16(ta + half * (DK / 2) + (2 * cb) * 16, w0);
+          tmem_st16(ta + half * (DK / 2) + (2 * cb + 1) * 16, w1);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sready[j]);
+        if (lane == 0) mbar_arrive(sready);
+      }
+      // c0_p = k_p . q_p for the epilogue (fp32 sums of the staged bf16 rows): thread
+      // (p, quarter) of the 128 coefficient threads takes a quarter of the row, then the four
+      // partial sums are added across lanes; SC[ac] is free once the epilogue of unit i - NA is
+      // done.
+      if (i >= NA) ok = ok && mbar_wait_bounded(&acc_empty[ac], ((i - NA) / NA) & 1);
+      {
+        const int tc = 32 * sp + lane, p = tc >> 2, qd = tc & 3;
+        const unsigned char* xs = stage(s);
+        float c0 = 0.f;
+#pragma unroll
+        for (int j = 0; j < CR / 4; ++j) {
+          const int c = qd * (CR / 4) + j, ks = c >> 3, cc = c & 7;
+          const uint4 qv = *reinterpret_cast<const uint4*>(xs + ks * 8192 + p * 128 + ((cc ^ (p & 7)) << 4));
+          const uint4 kv = *reinterpret_cast<const uint4*>(xs + ks * 8192 + (NP + p) * 128 +
+                                                           ((cc ^ ((NP + p) & 7)) << 4));
+          const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w}, kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw[e2]));
+            const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw[e2]));
+            c0 = fmaf(qf.x, kf.x, c0);
+            c0 = fmaf(qf.y, kf.y, c0);
+          }
+        }
+        c0 += __shfl_xor_sync(kFull, c0, 1);
+        c0 += __shfl_xor_sync(kFull, c0, 2);
+        if (qd == 0) SC[ac * NP + p].c0 = c0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&scal_ready[ac]);
       }
       // the decay table (always waited, so these warps never run two units ahead of the prep
       // warp), G, and the previous unit's MMAs (waited at every unit so that the wait never
       // falls two phases behind the barrier)
-      ok = ok && mbar_wait_bounded(&dec_ready[ac], (i >> 1) & 1);
+      ok = ok && mbar_wait_bounded(&dec_ready[ac], (i / NA) & 1);
       if (U > 0) {
         ok = ok && mbar_wait_bounded(g_ready, gcnt & 1);
         ++gcnt;
@@ -642,10 +629,11 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     const int row = 32 * sp + lane;
     const uint32_t tl = tmem + (uint32_t(32 * sp) << 16);
     __nv_bfloat16* Wb = reinterpret_cast<__nv_bfloat16*>(a.W);
+    __nv_bfloat16* kout = static_cast<__nv_bfloat16*>(a.Kr);
     for (int i = 0; i < n_my; ++i) {
-      const int s = i % NS, ac = i & 1;
-      bool ok = mbar_wait_bounded(&acc_full[ac], (i >> 1) & 1);
-      ok = ok && mbar_wait_bounded(&scal_ready[ac], (i >> 1) & 1);
+      const int s = i % NS, ac = i % NA;
+      bool ok = mbar_wait_bounded(&acc_full[ac], (i / NA) & 1);
+      ok = ok && mbar_wait_bounded(&scal_ready[ac], (i / NA) & 1);
       if (!__all_sync(kFull, ok)) {
         if (lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 26, t);
         break;
@@ -655,6 +643,20 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       const unsigned char* Vb = stage(s) + L.v_off;   // [2][32][128 B] sw128
       const MmaInfo* inf = info(s);
       const int n_pos = min(inf->n_pos, NP), U = inf->U;
+      // append k_p: the 256 epilogue threads copy the staged k rows (16-byte chunks)
+      {
+        const unsigned char* xs = stage(s);
+        const int e = ew * 32 + lane;
+#pragma unroll
+        for (int j = 0; j < CR / 8; ++j) {
+          const int idx = e * (CR / 8) + j, p = idx / CR, c = idx % CR, nn = NP + p;
+          if (p < n_pos) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xs + (c >> 3) * 8192 + nn * 128 +
+                                                            (((c & 7) ^ (nn & 7)) << 4));
+            *reinterpret_cast<uint4*>(kout + size_t(sc[p].wnew) * DK + c * 8) = v;
+          }
+        }
+      }
       const uint32_t base = tl + uint32_t(ac) * 128u;
 #pragma unroll 1
       for (int pb = 0; pb < 2; ++pb) {
