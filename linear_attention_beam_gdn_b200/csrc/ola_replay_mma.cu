@@ -22,14 +22,15 @@
 //
 // One CTA per SM walks the units of its (request, head) pairs, dealt round-robin, through a
 // three-stage ring. Warp roles:
-//   warps 0-2, 4-6  producers: TMA row gathers (tile::gather4, 128-byte swizzle) of the unit's
+//   warps 0-2, 4-5  producers: TMA row gathers (tile::gather4, 128-byte swizzle) of the unit's
 //               q, k and v rows, distinct ancestor keys and w records (the latter as the
-//               MN-major operand), one list of copies dealt out in six chunks; cp.async of the
-//               per-position scalars.
-//   warp 3      MMA: G with the staged q, k tile as A and the ancestor keys as B; D1 with S_ctx
-//               (bf16 hi + lo) held in tensor memory as the A operand; D2 with the staged w
-//               planes as the A operand and Cf as B, written over G. Three accumulator stages;
-//               D2 of unit i - 1 is issued before G and D1 of unit i.
+//               MN-major operand), one list of copies dealt out in five chunks; cp.async of
+//               the per-position scalars.
+//   warp 3      head MMA: G with the staged q, k tile as A and the ancestor keys as B; D1 with
+//               S_ctx (bf16 hi + lo) held in tensor memory as the A operand. Three accumulator
+//               stages.
+//   warp 6      tail MMA: D2 with the staged w planes as the A operand and Cf as B, written
+//               over G.
 //   warp 7      prep: decay table, per-position scalars, append of alpha_p.
 //   warps 8-11  coefficients: S_ctx into tensor memory when the (request, head) changes;
 //               k_p . q_p; Cf from G and the decay table.
@@ -47,19 +48,21 @@ constexpr int kMmaMaxB = 1024;
 constexpr int kMmaDV = 128;
 // A TMA instruction holds its warp for several hundred cycles plus roughly eighty per active
 // lane, while the instructions of different warps proceed in parallel: the copies of a unit are
-// spread over six producer warps, one warp-wide gather instruction each.
+// spread over five producer warps, one warp-wide gather instruction each.
+// Two warps issue tensor-core work: the head warp (G and D1 of a unit, as soon as its operands
+// and an accumulator stage are there) and the tail warp (D2 once Cf is written), so that the
+// tensor pipe is fed from both ends of the pipeline.
 // Warp w runs on subpartition w % 4. Every subpartition holds one coefficient warp and two
-// epilogue warps (their tensor-memory lane quarter is w % 4); the producers fill subpartitions
-// 0-2 and the MMA and prep warps share subpartition 3, so that each subpartition's warps run
-// few distinct loops (the instruction cache is small next to this kernel).
-constexpr int kMmaProd = 6, kMmaCoef = 4, kMmaEpi = 8;
-constexpr int kMmaWarps = kMmaProd + 2 + kMmaCoef + kMmaEpi;   // 20 warps, 5 per subpartition
-constexpr int kMmaWMma = 3;                     // subpartition 3
-constexpr int kMmaWPrep = 7;                    // subpartition 3
+// epilogue warps (their tensor-memory lane quarter is w % 4).
+constexpr int kMmaProd = 5, kMmaCoef = 4, kMmaEpi = 8;
+constexpr int kMmaWarps = kMmaProd + 3 + kMmaCoef + kMmaEpi;   // 20 warps, 5 per subpartition
+constexpr int kMmaWMma = 3;                     // head MMA warp
+constexpr int kMmaWTail = 6;                    // tail MMA warp
+constexpr int kMmaWPrep = 7;
 constexpr int kMmaWCoef = 8;                    // warps 8..11 (subpartitions 0..3)
 constexpr int kMmaWEpi = kMmaWCoef + kMmaCoef;  // warps 12..19
 static_assert(kMmaWCoef % 4 == 0 && kMmaWEpi % 4 == 0, "tensor-memory lane quarters follow warp % 4");
-static_assert(kMmaWCoef == kMmaProd + 2, "warps 0..7 are the producers, the MMA and the prep warp");
+static_assert(kMmaWCoef == kMmaProd + 3, "warps 0..7 are the producers, the MMA and the prep warps");
 
 // Record row of (step slot, request r, beam b, head h) in this kernel's record storage, which
 // keeps the heads of a beam next to each other: [T_max][R][B][H] (the heads of one beam are
@@ -126,19 +129,19 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
   const MmaLayout L = mma_layout(DK);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* full = bars;               // [NS] stage loaded: cp.async arrivals + 1, TMA bytes
-  uint64_t* empty = full + NS;         // [NS] stage consumed: MMA commit, prep warp, epilogue warps
-  uint64_t* acc_full = empty + NS;     // [NA] accumulators of a unit complete
+  uint64_t* empty = full + NS;         // [NS] stage consumed: 2 MMA commits, prep, epilogue warps
+  uint64_t* acc_full = empty + NS;     // [NA] accumulators of a unit complete (D1 and D2 commits)
   uint64_t* acc_empty = acc_full + NA; // [NA] epilogue done with an accumulator stage
   uint64_t* scal_ready = acc_empty + NA;  // [NA] per-position scalars written
   uint64_t* dec_ready = scal_ready + NA;  // [NA] decay table buffer written
   uint64_t* dec_free = dec_ready + NA;    // [NA] coefficient warps done with a decay table buffer
   uint64_t* coef_ready = dec_free + NA;   // Cf of the current unit written (every unit)
-  uint64_t* coef_free = coef_ready + 1;   // MMAs of the previous unit done (Cf may be rewritten)
+  uint64_t* coef_free = coef_ready + 1;   // D2 of the previous unit done (Cf may be rewritten)
   uint64_t* sready = coef_free + 1;    // S_ctx loaded into tensor memory
   uint64_t* sfree = sready + 1;        // last MMA reading S_ctx done
-  uint64_t* g_ready = sfree + 1;       // G of the current unit in tensor memory (units with U > 0)
-  uint32_t* holder = reinterpret_cast<uint32_t*>(g_ready + 1);
-  static_assert((2 * NS + 5 * NA + 5) * 8 + 8 <= 256, "barrier area");
+  uint64_t* g_ready = sfree + 1;       // [NA] G of a unit in tensor memory (every unit)
+  uint32_t* holder = reinterpret_cast<uint32_t*>(g_ready + NA);
+  static_assert((2 * NS + 6 * NA + 4) * 8 + 8 <= 256, "barrier area");
   auto stage = [&](int s) { return smem + size_t(s) * L.stage; };
   auto info = [&](int s) { return reinterpret_cast<MmaInfo*>(stage(s) + L.info_off); };
   unsigned char* CH = smem + L.ch_off;
@@ -157,10 +160,11 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 32 * kMmaProd + 1);   // cp.async arrivals + header (with bytes)
-      mbar_init(&empty[s], 1 + 1 + kMmaEpi);
+      mbar_init(&empty[s], 2 + 1 + kMmaEpi);
     }
     for (int x = 0; x < NA; ++x) {
-      mbar_init(&acc_full[x], 1);
+      mbar_init(&acc_full[x], 2);
+      mbar_init(&g_ready[x], 1);
       mbar_init(&acc_empty[x], kMmaEpi);
       mbar_init(&scal_ready[x], 1 + kMmaCoef);   // prep warp, c0 from the coefficient warps
       mbar_init(&dec_ready[x], 1);
@@ -170,7 +174,6 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     mbar_init(coef_free, 1);
     mbar_init(sready, kMmaCoef);
     mbar_init(sfree, 1);
-    mbar_init(g_ready, 1);
     fence_barrier_init();
   }
   if (warp == kMmaWMma) tmem_alloc(holder, 512);
@@ -184,9 +187,9 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
   // D2 k), [384, 512) S_ctx (hi in the first d_k / 2 columns, lo after)
   const uint32_t tmem = *holder;
 
-  if (warp < kMmaWCoef && warp != kMmaWMma && warp != kMmaWPrep) {
+  if (warp < kMmaWCoef && warp != kMmaWMma && warp != kMmaWTail && warp != kMmaWPrep) {
     // ------------------------------------------------------------------ producers
-    const int pw = warp < kMmaWMma ? warp : warp - 1;     // 0..5
+    const int pw = warp < kMmaWMma ? warp : warp - 1;     // 0..4
     int issued = 0;
     if (n_my > 0) {
       int r = int(blockIdx.x) / a.H, h = int(blockIdx.x) % a.H, k = 0;
@@ -280,7 +283,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           __syncwarp();
         }
         {
-          const int C = (nops + kMmaProd - 1) / kMmaProd;          // <= 20 (<= 120 copies)
+          const int C = (nops + kMmaProd - 1) / kMmaProd;          // <= 24 (<= 120 copies)
           const int id = pw * C + lane;
           const bool has = lane < C && id < nops;
           const int kind = id < nqk ? 0 : id < nqk + nv ? 1 : id < nqk + nv + nka ? 2 : 3;
@@ -346,55 +349,28 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     for (int i = issued > NS ? issued - NS : 0; i < issued; ++i)
       mbar_wait_bounded(&full[i % NS], (i / NS) & 1);
   } else if (warp == kMmaWMma) {
-    // ------------------------------------------------------------------ MMA (whole warp)
-    // The warp runs converged; one elected lane issues each tensor-core instruction.
-    // Software-pipelined by one unit: iteration i first finishes unit i - 1 (D2 once its Cf is
-    // written, then the commits that hand it to the epilogue), then starts unit i (G, D1). The
-    // coefficient warps build Cf of unit i while the tensor pipe runs unit i's D1 and the
-    // epilogue drains unit i - 1.
-    int sver = -1, last_i = -1;
-    int pU = 0, ps = 0, pac = 0, plast = 0;             // the unit whose D2 is pending
+    // ------------------------------------------------------------------ head MMA warp
+    // The warp runs converged; one elected lane issues each tensor-core instruction. Per unit:
+    // G (into the D2 columns of the unit's accumulator stage), then D1.
+    int sver = -1;
     bool ok = true;
-    for (int i = 0; i <= n_my && ok; ++i) {
-      if (i >= 1) {
-        ok = __all_sync(kFull, mbar_wait_bounded(coef_ready, (i - 1) & 1));
-        tc_fence_after();
-        if (ok) {
-          const uint32_t d2 = tmem + uint32_t(pac) * 128u + 64u;
-          const uint32_t st = smem_u32(stage(ps));
-          const uint32_t id2 = idesc_bf16_f32_amn(128, 2 * NP);
-#pragma unroll 1
-          for (int kq = 0; kq < (pU + 15) / 16; ++kq) {
-            const uint64_t ah = sw128_mnmajor_desc(st + L.wh_off + kq * 4096, 1024, 2048);
-            const uint64_t al = sw128_mnmajor_desc(st + L.wl_off + kq * 4096, 1024, 2048);
-            const uint64_t bh = sw128_kmajor_desc(smem_u32(CH) + kq * 32);
-            const uint64_t bl = sw128_kmajor_desc(smem_u32(CL) + kq * 32);
-            umma_bf16_w(d2, ah, bh, id2, kq != 0 ? 1u : 0u);
-            umma_bf16_w(d2, al, bh, id2, 1u);
-            umma_bf16_w(d2, ah, bl, id2, 1u);
-          }
-          umma_commit_w(&acc_full[pac]);
-          umma_commit_w(coef_free);
-          umma_commit_w(&empty[ps]);
-          if (plast) umma_commit_w(sfree);
-          last_i = i - 1;
-        }
-      }
-      if (ok && i < n_my) {
-        const int s = i % NS, n = i / NS, ac = i % NA;
-        ok = __all_sync(kFull, mbar_wait_bounded(&full[s], n & 1));
-        fence_proxy_async_smem();                  // cp.async data -> tensor-core reads
-        const MmaInfo* inf = info(s);
-        const int U = min(inf->U, UC);
-        if (inf->first) ++sver;
-        if (i >= NA) ok = ok && __all_sync(kFull, mbar_wait_bounded(&acc_empty[ac], ((i - NA) / NA) & 1));
-        tc_fence_after();
-        const uint32_t d1 = tmem + uint32_t(ac) * 128u, d2 = d1 + 64u;
-        const uint32_t st = smem_u32(stage(s));
-        if (ok && U > 0) {
-          // G[x][u] = x . k_u (M = 64 rows x of the q | k tile, N = 48 records), into the
-          // columns that D2 overwrites once the coefficient warps have read G
-          const uint32_t id0 = idesc_bf16_f32(64, UC);
+    for (int i = 0; i < n_my && ok; ++i) {
+      const int s = i % NS, n = i / NS, ac = i % NA;
+      ok = __all_sync(kFull, mbar_wait_bounded(&full[s], n & 1));
+      fence_proxy_async_smem();                    // cp.async data -> tensor-core reads
+      const MmaInfo* inf = info(s);
+      const int U = min(inf->U, UC);
+      const int lastu = inf->last;
+      if (inf->first) ++sver;
+      if (i >= NA) ok = ok && __all_sync(kFull, mbar_wait_bounded(&acc_empty[ac], ((i - NA) / NA) & 1));
+      tc_fence_after();
+      const uint32_t d1 = tmem + uint32_t(ac) * 128u, d2 = d1 + 64u;
+      const uint32_t st = smem_u32(stage(s));
+      if (ok) {
+        // G[x][u] = x . k_u (M = 64 rows x of the q | k tile, N = 48 records), into the
+        // columns that D2 overwrites once the coefficient warps have read G
+        const uint32_t id0 = idesc_bf16_f32(64, UC);
+        if (U > 0) {
 #pragma unroll 1
           for (int kstep = 0; kstep < DK / 16; ++kstep) {
             const uint32_t ks = uint32_t(kstep >> 2), kk = uint32_t(kstep & 3);
@@ -402,30 +378,61 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
             const uint64_t bk = sw128_kmajor_desc(st + L.ka_off + ks * (UC * 128u) + kk * 32u);
             umma_bf16_w(d2, ax, bk, id0, kstep != 0 ? 1u : 0u);
           }
-          umma_commit_w(g_ready);
         }
-        ok = ok && __all_sync(kFull, mbar_wait_bounded(sready, sver & 1));
-        tc_fence_after();
-        if (ok) {
-          const uint32_t sa = tmem + 128u * NA;
-          const uint32_t id1 = idesc_bf16_f32(128, 2 * NP);
+        umma_commit_w(&g_ready[ac]);
+      }
+      ok = ok && __all_sync(kFull, mbar_wait_bounded(sready, sver & 1));
+      tc_fence_after();
+      if (ok) {
+        const uint32_t sa = tmem + 128u * NA;
+        const uint32_t id1 = idesc_bf16_f32(128, 2 * NP);
 #pragma unroll 1
-          for (int kstep = 0; kstep < DK / 16; ++kstep) {
-            const uint32_t ks = uint32_t(kstep >> 2), kk = uint32_t(kstep & 3);
-            const uint64_t bx = sw128_kmajor_desc(st + ks * 8192u + kk * 32u);
-            umma_bf16_ts_w(d1, sa + kstep * 8, bx, id1, kstep != 0 ? 1u : 0u);
-            umma_bf16_ts_w(d1, sa + DK / 2 + kstep * 8, bx, id1, 1u);
-          }
+        for (int kstep = 0; kstep < DK / 16; ++kstep) {
+          const uint32_t ks = uint32_t(kstep >> 2), kk = uint32_t(kstep & 3);
+          const uint64_t bx = sw128_kmajor_desc(st + ks * 8192u + kk * 32u);
+          umma_bf16_ts_w(d1, sa + kstep * 8, bx, id1, kstep != 0 ? 1u : 0u);
+          umma_bf16_ts_w(d1, sa + DK / 2 + kstep * 8, bx, id1, 1u);
         }
-        pU = U;
-        ps = s;
-        pac = ac;
-        plast = inf->last;
+        // S_ctx is read by D1 only: after the last unit of a (request, head) it may be replaced
+        if (lastu) umma_commit_w(sfree);
+        umma_commit_w(&empty[s]);
+        umma_commit_w(&acc_full[ac]);
       }
       if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 21, t);
     }
-    // tensor memory is released only once the last MMA has completed
-    if (last_i >= 0) mbar_wait_bounded(&acc_full[last_i % NA], (last_i / NA) & 1);
+    // tensor memory is released only once the last MMAs have completed
+    if (ok && n_my > 0) mbar_wait_bounded(&acc_full[(n_my - 1) % NA], ((n_my - 1) / NA) & 1);
+    __syncwarp();
+  } else if (warp == kMmaWTail) {
+    // ------------------------------------------------------------------ tail MMA warp
+    // Per unit, once its Cf is written: D2 = W^T Cf over the G columns.
+    bool ok = true;
+    for (int i = 0; i < n_my && ok; ++i) {
+      const int s = i % NS, ac = i % NA;
+      ok = __all_sync(kFull, mbar_wait_bounded(coef_ready, i & 1));
+      tc_fence_after();
+      if (ok) {
+        const int U = min(info(s)->U, UC);
+        const uint32_t d2 = tmem + uint32_t(ac) * 128u + 64u;
+        const uint32_t st = smem_u32(stage(s));
+        const uint32_t id2 = idesc_bf16_f32_amn(128, 2 * NP);
+#pragma unroll 1
+        for (int kq = 0; kq < (U + 15) / 16; ++kq) {
+          const uint64_t ah = sw128_mnmajor_desc(st + L.wh_off + kq * 4096, 1024, 2048);
+          const uint64_t al = sw128_mnmajor_desc(st + L.wl_off + kq * 4096, 1024, 2048);
+          const uint64_t bh = sw128_kmajor_desc(smem_u32(CH) + kq * 32);
+          const uint64_t bl = sw128_kmajor_desc(smem_u32(CL) + kq * 32);
+          umma_bf16_w(d2, ah, bh, id2, kq != 0 ? 1u : 0u);
+          umma_bf16_w(d2, al, bh, id2, 1u);
+          umma_bf16_w(d2, ah, bl, id2, 1u);
+        }
+        umma_commit_w(coef_free);
+        umma_commit_w(&empty[s]);
+        umma_commit_w(&acc_full[ac]);
+      }
+      if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 24, t);
+    }
+    if (ok && n_my > 0) mbar_wait_bounded(&acc_full[(n_my - 1) % NA], ((n_my - 1) / NA) & 1);
     __syncwarp();
   } else if (warp == kMmaWPrep) {
     // ------------------------------------------------------------------ prep warp
@@ -497,7 +504,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
   } else if (warp < kMmaWEpi) {
     // ------------------------------------------------------------------ coefficient warps
     const int sp = warp & 3;
-    int sver = -1, gcnt = 0;
+    int sver = -1;
     for (int i = 0; i < n_my; ++i) {
       const int s = i % NS, n = i / NS, ac = i % NA;
       bool ok = mbar_wait_bounded(&full[s], n & 1);
@@ -565,10 +572,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       // warp), G, and the previous unit's MMAs (waited at every unit so that the wait never
       // falls two phases behind the barrier)
       ok = ok && mbar_wait_bounded(&dec_ready[ac], (i / NA) & 1);
-      if (U > 0) {
-        ok = ok && mbar_wait_bounded(g_ready, gcnt & 1);
-        ++gcnt;
-      }
+      ok = ok && mbar_wait_bounded(&g_ready[ac], (i / NA) & 1);
       if (i >= 1) ok = ok && mbar_wait_bounded(coef_free, (i - 1) & 1);
       if (!__all_sync(kFull, ok)) {
         if (lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 25, t);
