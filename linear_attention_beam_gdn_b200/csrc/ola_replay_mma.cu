@@ -21,7 +21,7 @@
 // split of Henry, Tang & Heinecke 2019).
 //
 // One CTA per SM walks the units of its (request, head) pairs, dealt round-robin, through a
-// three-stage ring. Warp roles:
+// three-stage operand ring and a four-slot ring of v rows and unit headers. Warp roles:
 //   warps 0-2, 4-5  producers: TMA row gathers (tile::gather4, 128-byte swizzle) of the unit's
 //               q, k and v rows, distinct ancestor keys and w records (the latter as the
 //               MN-major operand), one list of copies dealt out in five chunks; cp.async of
@@ -33,15 +33,16 @@
 //               over G.
 //   warp 7      prep: decay table, per-position scalars, append of alpha_p.
 //   warps 8-11  coefficients: S_ctx into tensor memory when the (request, head) changes;
-//               k_p . q_p; Cf from G and the decay table.
+//               k_p . q_p and the append of k_p; Cf from G and the decay table.
 //   warps 12-19 epilogue: thread = state row i; w_p[i] and o_p[i] from D1, D2 and the scalars;
-//               stores o (fp32), the w record (hi, lo) and the k_p record.
+//               stores o (fp32) and the w record (hi, lo).
 // Every wait is bounded; on timeout the kernel records OLA_ERR_TIMEOUT and finishes.
 #include "ola_device.cuh"
 
 namespace ola {
 
-constexpr int kMmaStages = 3;    // operand stages in shared memory
+constexpr int kMmaStages = 3;    // operand stages in shared memory (q / k tile, keys, w planes)
+constexpr int kMmaVSlots = 4;    // v / unit-header slots (held until the epilogue is done)
 constexpr int kMmaAcc = 3;       // accumulator stages in tensor memory (and scalar / decay buffers)
 constexpr int kMmaMaxT = 12;
 constexpr int kMmaMaxB = 1024;
@@ -85,15 +86,18 @@ struct MmaScal {                 // per position
   int io, wnew, valid, pad;
 };
 
-// Shared memory (every tile 1024-byte aligned):
-//   stage s: X [NSL][64 rows: q of positions 0-31 | k of positions 0-31][128 B]  K-major, sw128
-//            KA [NSL][48 rows][128 B]       ancestor keys, same swizzle
-//            WH, WL [6 groups of 8 records][2 halves of d_v][8][128 B]  MN-major, sw128
-//            V [2 halves of d_v][32 positions][128 B]  sw128, MmaInfo
-//   then CH, CL [64 rows][128 B] (Cf hi, lo; K-major, sw128), DEC [3][32][48] fp32,
-//   SC [3][32], barriers.
+// Shared memory (every tile 1024-byte aligned). The operand stages are released once the
+// unit's MMAs and the coefficient warps are done with them; the v slots and unit headers, read
+// by the epilogue, live in a deeper ring of their own.
+//   operand stage s < 3: X [NSL][64 rows: q of positions 0-31 | k of positions 0-31][128 B]
+//                          K-major, sw128
+//                        KA [NSL][48 rows][128 B]   ancestor keys, same swizzle
+//                        WH, WL [6 groups of 8 records][2 halves of d_v][8][128 B]  MN-major
+//   v slot b < 4: V [2 halves of d_v][32 positions][128 B]  sw128
+//   MmaInfo [4], then CH, CL [64 rows][128 B] (Cf hi, lo; K-major, sw128), DEC [2][32][48]
+//   fp32, SC [3][32], barriers.
 struct MmaLayout {
-  uint32_t ka_off, wh_off, wl_off, v_off, info_off, stage;
+  uint32_t ka_off, wh_off, wl_off, stage, v_off, info_off;
   uint32_t ch_off, cl_off, dec_off, sc_off, bar_off, bytes;
 };
 
@@ -103,15 +107,15 @@ __host__ __device__ inline MmaLayout mma_layout(int d_k) {
   L.ka_off = NSL * 8192u;
   L.wh_off = L.ka_off + NSL * uint32_t(kUnitAnc) * 128u;
   L.wl_off = L.wh_off + uint32_t(kUnitAnc / 8) * 2048u;
-  L.v_off = L.wl_off + uint32_t(kUnitAnc / 8) * 2048u;
-  L.info_off = L.v_off + uint32_t(kUnitPos) * kMmaDV * 2u;
-  L.stage = (L.info_off + uint32_t(sizeof(MmaInfo)) + 1023u) & ~1023u;
-  L.ch_off = uint32_t(kMmaStages) * L.stage;
+  L.stage = L.wl_off + uint32_t(kUnitAnc / 8) * 2048u;
+  L.v_off = uint32_t(kMmaStages) * L.stage;
+  L.info_off = L.v_off + uint32_t(kMmaVSlots) * kUnitPos * kMmaDV * 2u;
+  L.ch_off = (L.info_off + uint32_t(kMmaVSlots) * uint32_t(sizeof(MmaInfo)) + 1023u) & ~1023u;
   L.cl_off = L.ch_off + 8192u;
   L.dec_off = L.cl_off + 8192u;
-  L.sc_off = L.dec_off + uint32_t(kMmaAcc) * kUnitPos * kUnitAnc * 4u;
+  L.sc_off = L.dec_off + 2u * kUnitPos * kUnitAnc * 4u;
   L.bar_off = L.sc_off + uint32_t(kMmaAcc) * kUnitPos * uint32_t(sizeof(MmaScal));
-  L.bytes = L.bar_off + 256u + 1024u;
+  L.bytes = L.bar_off + 320u + 1024u;
   return L;
 }
 
@@ -121,32 +125,36 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
                   StepArgs a, UnitPlan up, const __grid_constant__ CUtensorMap mq,
                   const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                   const __grid_constant__ CUtensorMap mkr, const __grid_constant__ CUtensorMap mw) {
-  constexpr int NS = kMmaStages, NA = kMmaAcc, DV = kMmaDV, UC = kUnitAnc, NP = kUnitPos;
+  constexpr int NS = kMmaStages, NB = kMmaVSlots, NA = kMmaAcc, DV = kMmaDV, UC = kUnitAnc,
+                NP = kUnitPos;
   constexpr int CR = DK / 8;       // 16-byte chunks of a key row
   constexpr int NSL = DK / 64;     // 64-column slices of a key row
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = align_smem_1024(smem_raw);
   const MmaLayout L = mma_layout(DK);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* full = bars;               // [NS] stage loaded: cp.async arrivals + 1, TMA bytes
-  uint64_t* empty = full + NS;         // [NS] stage consumed: 2 MMA commits, prep, epilogue warps
-  uint64_t* acc_full = empty + NS;     // [NA] accumulators of a unit complete (D1 and D2 commits)
+  uint64_t* fullA = bars;              // [NS] operand stage loaded: header arrive + TMA bytes
+  uint64_t* emptyA = fullA + NS;       // [NS] operand stage consumed: 2 MMA commits, coef warps
+  uint64_t* fullB = emptyA + NS;       // [NB] v slot and header loaded: cp.async arrivals + 1, bytes
+  uint64_t* emptyB = fullB + NB;       // [NB] v slot consumed: epilogue warps
+  uint64_t* acc_full = emptyB + NB;    // [NA] accumulators of a unit complete (D1 and D2 commits)
   uint64_t* acc_empty = acc_full + NA; // [NA] epilogue done with an accumulator stage
   uint64_t* scal_ready = acc_empty + NA;  // [NA] per-position scalars written
-  uint64_t* dec_ready = scal_ready + NA;  // [NA] decay table buffer written
-  uint64_t* dec_free = dec_ready + NA;    // [NA] coefficient warps done with a decay table buffer
-  uint64_t* coef_ready = dec_free + NA;   // Cf of the current unit written (every unit)
+  uint64_t* g_ready = scal_ready + NA;    // [NA] G of a unit in tensor memory (every unit)
+  uint64_t* dec_ready = g_ready + NA;     // [2] decay table buffer written
+  uint64_t* dec_free = dec_ready + 2;     // [2] coefficient warps done with a decay table buffer
+  uint64_t* coef_ready = dec_free + 2;    // Cf of the current unit written (every unit)
   uint64_t* coef_free = coef_ready + 1;   // D2 of the previous unit done (Cf may be rewritten)
   uint64_t* sready = coef_free + 1;    // S_ctx loaded into tensor memory
   uint64_t* sfree = sready + 1;        // last MMA reading S_ctx done
-  uint64_t* g_ready = sfree + 1;       // [NA] G of a unit in tensor memory (every unit)
-  uint32_t* holder = reinterpret_cast<uint32_t*>(g_ready + NA);
-  static_assert((2 * NS + 6 * NA + 4) * 8 + 8 <= 256, "barrier area");
+  uint32_t* holder = reinterpret_cast<uint32_t*>(sfree + 1);
+  static_assert((2 * NS + 2 * NB + 4 * NA + 8) * 8 + 8 <= 320, "barrier area");
   auto stage = [&](int s) { return smem + size_t(s) * L.stage; };
-  auto info = [&](int s) { return reinterpret_cast<MmaInfo*>(stage(s) + L.info_off); };
+  auto vslot = [&](int b) { return smem + L.v_off + size_t(b) * (NP * DV * 2); };
+  auto info = [&](int b) { return reinterpret_cast<MmaInfo*>(smem + L.info_off) + b; };
   unsigned char* CH = smem + L.ch_off;
   unsigned char* CL = smem + L.cl_off;
-  float* DEC0 = reinterpret_cast<float*>(smem + L.dec_off);   // [NA][32][48]
+  float* DEC0 = reinterpret_cast<float*>(smem + L.dec_off);   // [2][32][48]
   MmaScal* SC = reinterpret_cast<MmaScal*>(smem + L.sc_off);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -159,14 +167,20 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 32 * kMmaProd + 1);   // cp.async arrivals + header (with bytes)
-      mbar_init(&empty[s], 2 + 1 + kMmaEpi);
+      mbar_init(&fullA[s], 1);                  // expect-tx arrival (with the bytes)
+      mbar_init(&emptyA[s], 2 + kMmaCoef);
+    }
+    for (int b = 0; b < NB; ++b) {
+      mbar_init(&fullB[b], 32 * kMmaProd + 1);  // cp.async arrivals + header (with bytes)
+      mbar_init(&emptyB[b], kMmaEpi);
     }
     for (int x = 0; x < NA; ++x) {
       mbar_init(&acc_full[x], 2);
       mbar_init(&g_ready[x], 1);
       mbar_init(&acc_empty[x], kMmaEpi);
       mbar_init(&scal_ready[x], 1 + kMmaCoef);   // prep warp, c0 from the coefficient warps
+    }
+    for (int x = 0; x < 2; ++x) {
       mbar_init(&dec_ready[x], 1);
       mbar_init(&dec_free[x], kMmaCoef);
     }
@@ -177,7 +191,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     fence_barrier_init();
   }
   if (warp == kMmaWMma) tmem_alloc(holder, 512);
-  // zero the stages and the Cf tiles once: rows that no unit has filled yet hold finite values
+  // zero the stages, v slots and Cf tiles once: rows no unit has filled yet hold finite values
   for (uint32_t x = tid; x < L.dec_off / 16u; x += blockDim.x)
     reinterpret_cast<uint4*>(smem)[x] = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_smem();
@@ -199,8 +213,10 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       int x0 = __ldcg(rec + lane), x1 = __ldcg(rec + 32 + lane), x2 = __ldcg(rec + 64 + lane);
       int prev_rh = -1;
       for (int i = 0; i < n_my; ++i) {
-        const int s = i % NS, n = i / NS;
-        if (i >= NS && !__all_sync(kFull, mbar_wait_bounded(&empty[s], (n - 1) & 1))) {
+        const int s = i % NS, n = i / NS, sb = i % NB, nb = i / NB;
+        bool okw = i < NS || mbar_wait_bounded(&emptyA[s], (n - 1) & 1);
+        if (i >= NB) okw = okw && mbar_wait_bounded(&emptyB[sb], (nb - 1) & 1);
+        if (!__all_sync(kFull, okw)) {
           if (lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 20, t);
           break;
         }
@@ -229,9 +245,9 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         if (first) {
           // S_ctx hi/lo rows of this (request, head) (first unit only) and of the next one,
           // into L2 ahead of the builders' loads: 2 x 128 rows x 2 d_k bytes
-          const int nb = (prev_rh < 0 ? 2 : 1);
-          for (int q = 0; q < nb; ++q) {
-            const int rq = rh + (nb == 2 ? q : 1) * int(gridDim.x);
+          const int npf = (prev_rh < 0 ? 2 : 1);
+          for (int q = 0; q < npf; ++q) {
+            const int rq = rh + (npf == 2 ? q : 1) * int(gridDim.x);
             if (rq < a.R * a.H) {
               const unsigned char* hi_b = reinterpret_cast<const unsigned char*>(S_hi) + size_t(rq) * DV * DK * 2;
               const unsigned char* lo_b = reinterpret_cast<const unsigned char*>(S_lo) + size_t(rq) * DV * DK * 2;
@@ -258,12 +274,14 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         const int row0 = rec_row_hm(a, anc0 >> 16, r, h, anc0 & 0xffff);
         const int row1 = rec_row_hm(a, anc1 >> 16, r, h, anc1 & 0xffff);
         unsigned char* st = stage(s);
-        MmaInfo* inf = info(s);
+        unsigned char* vs = vslot(sb);
+        MmaInfo* inf = info(sb);
         // Every operand row goes in by TMA row gathers of four (tile::gather4, 128-byte
-        // swizzle, 64 columns per copy), all counted as transaction bytes on full[s]: q, k rows
-        // of the position groups, v rows, the ancestor keys and the w records (hi, lo x two
-        // halves of d_v). The copies form one list; warp pw issues entries [pw C, pw C + C) in
-        // one instruction. Rows past n_pos / U repeat row 0 (never read).
+        // swizzle, 64 columns per copy): q, k rows of the position groups, the ancestor keys
+        // and the w records (hi, lo x two halves of d_v) into the operand stage, counted as
+        // transaction bytes on fullA[s]; the v rows into the v slot, counted on fullB[sb]. The
+        // copies form one list; warp pw issues entries [pw C, pw C + C) in one instruction.
+        // Rows past n_pos / U repeat row 0 (never read).
         const int U4 = (U + 3) & ~3, G4 = (n_pos + 3) >> 2;
         const int nqk = 2 * G4 * NSL, nv = 2 * G4, nka = (U4 / 4) * NSL;
         const int nops = nqk + nv + nka + U4;
@@ -279,7 +297,10 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           }
           inf->beam[lane] = beam;
           __syncwarp();
-          if (lane == 0) mbar_arrive_expect_tx(&full[s], uint32_t(nops) * 512u);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&fullA[s], uint32_t(nops - nv) * 512u);
+            mbar_arrive_expect_tx(&fullB[sb], uint32_t(nv) * 512u);
+          }
           __syncwarp();
         }
         {
@@ -287,31 +308,34 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           const int id = pw * C + lane;
           const bool has = lane < C && id < nops;
           const int kind = id < nqk ? 0 : id < nqk + nv ? 1 : id < nqk + nv + nka ? 2 : 3;
-          int m, xc, sm_off;
+          int m, xc;
+          unsigned char* dst;
+          uint64_t* bar = &fullA[s];
           const CUtensorMap* map;
           if (kind == 0) {
             const int side = id >= G4 * NSL ? 1 : 0, e = id - side * G4 * NSL, ks = e % NSL;
             m = e / NSL;
             xc = 64 * ks;
-            sm_off = ks * 8192 + (side * NP + 4 * m) * 128;
+            dst = st + ks * 8192 + (side * NP + 4 * m) * 128;
             map = side ? &mk : &mq;
           } else if (kind == 1) {
             const int e = id - nqk, ks = e & 1;
             m = e >> 1;
             xc = 64 * ks;
-            sm_off = int(L.v_off) + ks * (NP * 128) + 4 * m * 128;
+            dst = vs + ks * (NP * 128) + 4 * m * 128;
+            bar = &fullB[sb];
             map = &mv;
           } else if (kind == 2) {
             const int e = id - nqk - nv, ks = e % NSL;
             m = e / NSL;
             xc = 64 * ks;
-            sm_off = int(L.ka_off) + ks * (UC * 128) + 4 * m * 128;
+            dst = st + L.ka_off + ks * (UC * 128) + 4 * m * 128;
             map = &mkr;
           } else {
             const int e = id - nqk - nv - nka, pl = (e >> 1) & 1, mb = e & 1;
             m = e >> 2;
             xc = 128 * pl + 64 * mb;
-            sm_off = int(pl ? L.wl_off : L.wh_off) + (4 * m >> 3) * 2048 + mb * 1024 + (4 * m & 7) * 128;
+            dst = st + (pl ? L.wl_off : L.wh_off) + (4 * m >> 3) * 2048 + mb * 1024 + (4 * m & 7) * 128;
             map = &mw;
           }
           int y[4];
@@ -323,7 +347,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
             const int rA = __shfl_sync(kFull, row0, uu & 31), rB = __shfl_sync(kFull, row1, uu & 31);
             y[j] = kind <= 1 ? yp : (uu < 32 ? rA : rB);
           }
-          if (has) tma_gather4(st + sm_off, map, &full[s], xc, y[0], y[1], y[2], y[3]);
+          if (has) tma_gather4(dst, map, bar, xc, y[0], y[1], y[2], y[3]);
         }
         if (pw == 1) {
           if (lane < n_pos) {
@@ -334,7 +358,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           if (lane < U) cp_async4(&inf->alpha[lane], a.A + row0);
           if (lane + 32 < U) cp_async4(&inf->alpha[32 + lane], a.A + row1);
         }
-        cp_async_arrive(&full[s]);
+        cp_async_arrive(&fullB[sb]);
         issued = i + 1;
         x0 = y0;
         x1 = y1;
@@ -347,7 +371,9 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     }
     // the CTA may not exit with copies in flight
     for (int i = issued > NS ? issued - NS : 0; i < issued; ++i)
-      mbar_wait_bounded(&full[i % NS], (i / NS) & 1);
+      mbar_wait_bounded(&fullA[i % NS], (i / NS) & 1);
+    for (int i = issued > NB ? issued - NB : 0; i < issued; ++i)
+      mbar_wait_bounded(&fullB[i % NB], (i / NB) & 1);
   } else if (warp == kMmaWMma) {
     // ------------------------------------------------------------------ head MMA warp
     // The warp runs converged; one elected lane issues each tensor-core instruction. Per unit:
@@ -355,10 +381,11 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     int sver = -1;
     bool ok = true;
     for (int i = 0; i < n_my && ok; ++i) {
-      const int s = i % NS, n = i / NS, ac = i % NA;
-      ok = __all_sync(kFull, mbar_wait_bounded(&full[s], n & 1));
+      const int s = i % NS, n = i / NS, sb = i % NB, ac = i % NA;
+      ok = __all_sync(kFull, mbar_wait_bounded(&fullA[s], n & 1) &&
+                                 mbar_wait_bounded(&fullB[sb], (i / NB) & 1));
       fence_proxy_async_smem();                    // cp.async data -> tensor-core reads
-      const MmaInfo* inf = info(s);
+      const MmaInfo* inf = info(sb);
       const int U = min(inf->U, UC);
       const int lastu = inf->last;
       if (inf->first) ++sver;
@@ -395,7 +422,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         }
         // S_ctx is read by D1 only: after the last unit of a (request, head) it may be replaced
         if (lastu) umma_commit_w(sfree);
-        umma_commit_w(&empty[s]);
+        umma_commit_w(&emptyA[s]);
         umma_commit_w(&acc_full[ac]);
       }
       if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 21, t);
@@ -412,7 +439,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       ok = __all_sync(kFull, mbar_wait_bounded(coef_ready, i & 1));
       tc_fence_after();
       if (ok) {
-        const int U = min(info(s)->U, UC);
+        const int U = min(info(i % NB)->U, UC);
         const uint32_t d2 = tmem + uint32_t(ac) * 128u + 64u;
         const uint32_t st = smem_u32(stage(s));
         const uint32_t id2 = idesc_bf16_f32_amn(128, 2 * NP);
@@ -427,7 +454,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           umma_bf16_w(d2, ah, bl, id2, 1u);
         }
         umma_commit_w(coef_free);
-        umma_commit_w(&empty[s]);
+        umma_commit_w(&emptyA[s]);
         umma_commit_w(&acc_full[ac]);
       }
       if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 24, t);
@@ -439,21 +466,18 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     // Per unit, from the staged data only (nothing here waits for a tensor-core result, so the
     // warp runs ahead): the decay table, the per-position scalars and the append of alpha_p.
     for (int i = 0; i < n_my; ++i) {
-      const int s = i % NS, n = i / NS, ac = i % NA;
-      bool ok = mbar_wait_bounded(&full[s], n & 1);
-      if (i >= NA) {
-        ok = ok && mbar_wait_bounded(&acc_empty[ac], ((i - NA) / NA) & 1);   // SC[ac] free
-        ok = ok && mbar_wait_bounded(&dec_free[ac], ((i - NA) / NA) & 1);    // DEC[ac] free
-      }
+      const int sb = i % NB, ac = i % NA, db = i & 1;
+      bool ok = mbar_wait_bounded(&fullB[sb], (i / NB) & 1);
+      if (i >= NA) ok = ok && mbar_wait_bounded(&acc_empty[ac], ((i - NA) / NA) & 1);  // SC[ac] free
+      if (i >= 2) ok = ok && mbar_wait_bounded(&dec_free[db], ((i - 2) >> 1) & 1);      // DEC[db] free
       if (!__all_sync(kFull, ok)) {
         if (lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 23, t);
         break;
       }
-      const MmaInfo* inf = info(s);
-      const unsigned char* st = stage(s);
+      const MmaInfo* inf = info(sb);
       const int r = inf->r, h = inf->h, n_pos = min(inf->n_pos, NP);
       MmaScal* sc = SC + ac * NP;
-      float* DEC = DEC0 + ac * (NP * UC);
+      float* DEC = DEC0 + db * (NP * UC);
       // position p = lane: beam, new record row, decay walk
       const int p = lane;
       const bool valid = p < n_pos;
@@ -496,19 +520,19 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       sc[p].valid = valid ? 1 : 0;
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&dec_ready[ac]);
+        mbar_arrive(&dec_ready[db]);
         mbar_arrive(&scal_ready[ac]);
-        mbar_arrive(&empty[s]);
       }
     }
   } else if (warp < kMmaWEpi) {
     // ------------------------------------------------------------------ coefficient warps
     const int sp = warp & 3;
     int sver = -1;
+    __nv_bfloat16* kout = static_cast<__nv_bfloat16*>(a.Kr);
     for (int i = 0; i < n_my; ++i) {
-      const int s = i % NS, n = i / NS, ac = i % NA;
-      bool ok = mbar_wait_bounded(&full[s], n & 1);
-      const MmaInfo* inf = info(s);
+      const int s = i % NS, n = i / NS, sb = i % NB, ac = i % NA, db = i & 1;
+      bool ok = mbar_wait_bounded(&fullA[s], n & 1) && mbar_wait_bounded(&fullB[sb], (i / NB) & 1);
+      const MmaInfo* inf = info(sb);
       const int r = inf->r, h = inf->h, U = min(inf->U, UC);
       if (inf->first) {
         ++sver;
@@ -565,13 +589,28 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         c0 += __shfl_xor_sync(kFull, c0, 1);
         c0 += __shfl_xor_sync(kFull, c0, 2);
         if (qd == 0) SC[ac * NP + p].c0 = c0;
+        // append k_p: the 128 threads copy the staged k rows (16-byte chunks) into the records
+        const int n_pos = min(inf->n_pos, NP);
+#pragma unroll
+        for (int j = 0; j < CR / 4; ++j) {
+          const int idx = tc * (CR / 4) + j, pk = idx / CR, c = idx % CR, nn = NP + pk;
+          if (pk < n_pos) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xs + (c >> 3) * 8192 + nn * 128 +
+                                                            (((c & 7) ^ (nn & 7)) << 4));
+            const int wr = rec_row_hm(a, t - 1, r, h, inf->beam[pk]);
+            *reinterpret_cast<uint4*>(kout + size_t(wr) * DK + c * 8) = v;
+          }
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&scal_ready[ac]);
+        if (lane == 0) {
+          mbar_arrive(&scal_ready[ac]);
+          mbar_arrive(&emptyA[s]);                   // done with the operand stage
+        }
       }
       // the decay table (always waited, so these warps never run two units ahead of the prep
       // warp), G, and the previous unit's MMAs (waited at every unit so that the wait never
       // falls two phases behind the barrier)
-      ok = ok && mbar_wait_bounded(&dec_ready[ac], (i / NA) & 1);
+      ok = ok && mbar_wait_bounded(&dec_ready[db], (i >> 1) & 1);
       ok = ok && mbar_wait_bounded(&g_ready[ac], (i / NA) & 1);
       if (i >= 1) ok = ok && mbar_wait_bounded(coef_free, (i - 1) & 1);
       if (!__all_sync(kFull, ok)) {
@@ -585,7 +624,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         // lanes 0-15 of subpartition sp).
         const uint32_t tg = tmem + (uint32_t(32 * sp) << 16) + uint32_t(ac) * 128u + 64u;
         const int nrow = 16 * sp + (lane & 15), p = nrow & 31;
-        const float* dr = DEC0 + ac * (NP * UC) + p * UC;
+        const float* dr = DEC0 + db * (NP * UC) + p * UC;
 #pragma unroll 1
         for (int h16 = 0; h16 < UC / 16; ++h16) {
           if (16 * h16 >= U) break;                   // warp-uniform
@@ -622,7 +661,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&dec_free[ac]);
+        mbar_arrive(&dec_free[db]);
         mbar_arrive(coef_ready);
       }
     }
@@ -633,9 +672,8 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     const int row = 32 * sp + lane;
     const uint32_t tl = tmem + (uint32_t(32 * sp) << 16);
     __nv_bfloat16* Wb = reinterpret_cast<__nv_bfloat16*>(a.W);
-    __nv_bfloat16* kout = static_cast<__nv_bfloat16*>(a.Kr);
     for (int i = 0; i < n_my; ++i) {
-      const int s = i % NS, ac = i % NA;
+      const int sb = i % NB, ac = i % NA;
       bool ok = mbar_wait_bounded(&acc_full[ac], (i / NA) & 1);
       ok = ok && mbar_wait_bounded(&scal_ready[ac], (i / NA) & 1);
       if (!__all_sync(kFull, ok)) {
@@ -644,23 +682,9 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       }
       tc_fence_after();
       const MmaScal* sc = SC + ac * NP;
-      const unsigned char* Vb = stage(s) + L.v_off;   // [2][32][128 B] sw128
-      const MmaInfo* inf = info(s);
+      const unsigned char* Vb = vslot(sb);          // [2][32][128 B] sw128
+      const MmaInfo* inf = info(sb);
       const int n_pos = min(inf->n_pos, NP), U = inf->U;
-      // append k_p: the 256 epilogue threads copy the staged k rows (16-byte chunks)
-      {
-        const unsigned char* xs = stage(s);
-        const int e = ew * 32 + lane;
-#pragma unroll
-        for (int j = 0; j < CR / 8; ++j) {
-          const int idx = e * (CR / 8) + j, p = idx / CR, c = idx % CR, nn = NP + p;
-          if (p < n_pos) {
-            const uint4 v = *reinterpret_cast<const uint4*>(xs + (c >> 3) * 8192 + nn * 128 +
-                                                            (((c & 7) ^ (nn & 7)) << 4));
-            *reinterpret_cast<uint4*>(kout + size_t(sc[p].wnew) * DK + c * 8) = v;
-          }
-        }
-      }
       const uint32_t base = tl + uint32_t(ac) * 128u;
 #pragma unroll 1
       for (int pb = 0; pb < 2; ++pb) {
@@ -713,7 +737,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&acc_empty[ac]);
-        mbar_arrive(&empty[s]);
+        mbar_arrive(&emptyB[sb]);
       }
     }
   }
