@@ -87,9 +87,10 @@ cudaError_t launch_plan(const StepArgs& a, cudaStream_t stream) {
 size_t plan_units_smem(int B, int T_max) {
   const int Bp = (B + 3) & ~3, TA = T_max > 1 ? T_max - 1 : 1;
   // keys, parents, perm, chains, change masks, unit of position, unit start/size/U, counts,
-  // sibling-group starts and sizes, scratch
+  // sibling-group starts and sizes, prefix sums of group sizes and new-record counts, unit
+  // ends, scratch
   return sizeof(int) * (size_t(Bp) + B + B + size_t(B) * TA + B + B + 3 * size_t(B) +
-                        size_t(B) * TA + 2 * size_t(B) + 64);
+                        size_t(B) * TA + 2 * size_t(B) + 3 * size_t(B + 1) + 128);
 }
 
 __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up) {
@@ -109,7 +110,10 @@ __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up
   int* sdist = uU + B;            // [B][TA] distinct records per (unit, slot)
   int* gst = sdist + B * TA;      // [B] start of each sibling group
   int* gsz = gst + B;             // [B] its size
-  int* misc = gsz + B;            // [0] unit count, [1] last-CTA flag, [2] groups, [32..] scratch
+  int* PS = gsz + B;              // [B + 1] prefix sums of the group sizes
+  int* PC = PS + (B + 1);         // [B + 1] prefix sums of the groups' new-record counts
+  int* gnext = PC + (B + 1);      // [B + 1] end (exclusive) of a unit starting at group g
+  int* misc = gnext + (B + 1);    // [0] unit count, [1] last-CTA flag, [2] groups, [32..] scratch
 
   // depth-first order: stable sort of the beams by their parent's position (ola_plan.cu above)
   for (int b = tid; b < Bp; b += nt) {
@@ -139,15 +143,26 @@ __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up
     sperm[pos] = b;
   }
   __syncthreads();
-  // parent chains by position; chain rows of the new beams
-  for (int x = tid; x < B * n_anc; x += nt) {
-    const int pos = x / n_anc, s = x % n_anc;
+  // parent chains by position; chain rows of the new beams (a thread per position: the parent's
+  // chain entries are all loaded before any is stored)
+  for (int pos = tid; pos < B; pos += nt) {
     const int b = sperm[pos];
-    const int c = a.C[chain_row(a, a.t - 2, r, pbuf[b]) + s];
-    spch[pos * TA + s] = c;
-    a.C[chain_row(a, a.t - 1, r, b) + s] = c;
+    int* dst = a.C + chain_row(a, a.t - 1, r, b);
+    for (int s0 = 0; s0 < n_anc; s0 += 8) {
+      const int* src = a.C + chain_row(a, a.t - 2, r, pbuf[b]) + s0;
+      int cv[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) cv[q] = s0 + q < n_anc ? src[q] : 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (s0 + q < n_anc) {
+          spch[pos * TA + s0 + q] = cv[q];
+          dst[s0 + q] = cv[q];
+        }
+      }
+    }
+    dst[n_anc] = b;
   }
-  for (int pos = tid; pos < B; pos += nt) a.C[chain_row(a, a.t - 1, r, sperm[pos]) + n_anc] = sperm[pos];
   __syncthreads();
   for (int pos = tid; pos < B; pos += nt) {
     int m = 0;
@@ -184,83 +199,126 @@ __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up
     for (int g = tid; g < carry; g += nt) gsz[g] = (g + 1 < carry ? gst[g + 1] : B) - gst[g];
   }
   __syncthreads();
-  // units (one warp). Beams with the same parent have the same chain, and their outputs must not
-  // depend on how the beams are cut into units: a unit holds whole sibling groups of at most
-  // kUnitPos positions while its distinct records stay <= kUnitAnc (greedy, left to right);
-  // a larger group is cut into chunks of kUnitPos positions, each a unit of its own, so that
-  // every chunk lists the chain's records in the same order (record u = chain slot u).
-  if (warp == 0) {
+  // units. Beams with the same parent have the same chain, and their outputs must not depend on
+  // how the beams are cut into units: a unit holds whole sibling groups of at most kUnitPos
+  // positions while its distinct records stay <= kUnitAnc (greedy, left to right); a larger
+  // group is cut into chunks of kUnitPos positions, each a unit of its own, so that every chunk
+  // lists the chain's records in the same order (record u = chain slot u). A unit starting at
+  // group g takes n_anc records for its first group and popc(fnew) new ones for each further
+  // group, so its end is found by binary search on prefix sums of the group sizes and of the
+  // new-record counts; one thread then follows the chain of unit starts.
+  {
     const int ng = misc[2];
-    int g0 = 0, k = 0;
-    while (g0 < ng) {
-      const int gs0 = gst[g0], sz0 = gsz[g0];
-      if (sz0 > kUnitPos) {
-        for (int off = 0; off < sz0; off += kUnitPos) {
-          const int n = min(kUnitPos, sz0 - off);
-          if (lane == 0) {
-            ustart[k] = gs0 + off;
-            un[k] = n;
-            uU[k] = n_anc;
-          }
-          if (lane < n) uop[gs0 + off + lane] = k;
-          ++k;
-        }
-        ++g0;
-        continue;
-      }
-      const int g = g0 + lane;
-      const bool gv = g < ng;
-      int S = gv ? gsz[g] : (1 << 20);
-      int C = gv ? (lane == 0 ? n_anc : __popc(fnew[gst[g]])) : (1 << 20);
-      const unsigned bad = __ballot_sync(kFull, !gv || S > kUnitPos);
+    int carry_s = 0, carry_c = 0;
+    for (int base = 0; base < ng; base += nt) {
+      const int g = base + tid;
+      const int s1 = g < ng ? gsz[g] : 0;
+      const int c1 = g < ng ? __popc(fnew[gst[g]]) : 0;
+      int xs = s1, xc = c1;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
-        const int ys = __shfl_up_sync(kFull, S, off), yc = __shfl_up_sync(kFull, C, off);
+        const int ys = __shfl_up_sync(kFull, xs, off), yc = __shfl_up_sync(kFull, xc, off);
         if (lane >= off) {
-          S += ys;
-          C += yc;
+          xs += ys;
+          xc += yc;
         }
       }
-      const int firstbad = bad ? __ffs(bad) - 1 : 32;
-      // S, C grow with the lane, so the accepted lanes are a prefix; lane 0 always fits
-      const unsigned m = __ballot_sync(kFull, lane < firstbad && S <= kUnitPos && C <= kUnitAnc);
-      const int ngr = __popc(m);
-      const int n = __shfl_sync(kFull, S, ngr - 1), U = __shfl_sync(kFull, C, ngr - 1);
-      if (lane == 0) {
-        ustart[k] = gs0;
-        un[k] = n;
-        uU[k] = U;
+      if (lane == 31) {
+        misc[32 + warp] = xs;
+        misc[64 + warp] = xc;
       }
-      if (lane < n) uop[gs0 + lane] = k;
-      ++k;
-      g0 += ngr;
+      __syncthreads();
+      int bs = 0, bc = 0, ts = 0, tcn = 0;
+      for (int w2 = 0; w2 < nt / 32; ++w2) {
+        if (w2 < warp) {
+          bs += misc[32 + w2];
+          bc += misc[64 + w2];
+        }
+        ts += misc[32 + w2];
+        tcn += misc[64 + w2];
+      }
+      if (g < ng) {
+        PS[g + 1] = carry_s + bs + xs;
+        PC[g + 1] = carry_c + bc + xc;
+      }
+      carry_s += ts;
+      carry_c += tcn;
+      __syncthreads();
     }
-    if (lane == 0) misc[0] = k;
+    if (tid == 0) {
+      PS[0] = 0;
+      PC[0] = 0;
+    }
+    __syncthreads();
+    for (int g = tid; g < ng; g += nt) {
+      // smallest j in (g, ng] at which adding group j breaks a limit (a group larger than
+      // kUnitPos breaks the size limit by itself)
+      int lo = g + 1, hi = ng;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const bool viol = PS[mid + 1] - PS[g] > kUnitPos || n_anc + PC[mid + 1] - PC[g + 1] > kUnitAnc;
+        if (viol) hi = mid;
+        else lo = mid + 1;
+      }
+      gnext[g] = lo;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int g = 0, k = 0;
+      while (g < ng) {
+        const int gs0 = gst[g], sz0 = gsz[g];
+        if (sz0 > kUnitPos) {
+          for (int off = 0; off < sz0; off += kUnitPos) {
+            ustart[k] = gs0 + off;
+            un[k] = min(kUnitPos, sz0 - off);
+            uU[k] = n_anc;
+            ++k;
+          }
+          ++g;
+          continue;
+        }
+        const int j = gnext[g];
+        ustart[k] = gs0;
+        un[k] = PS[j] - PS[g];
+        uU[k] = n_anc + PC[j] - PC[g + 1];
+        ++k;
+        g = j;
+      }
+      misc[0] = k;
+    }
+    __syncthreads();
+    const int nu0 = misc[0];
+    for (int x = tid; x < nu0 * kUnitPos; x += nt) {
+      const int k = x / kUnitPos, j = x % kUnitPos;
+      if (j < un[k]) uop[ustart[k] + j] = k;
+    }
   }
   __syncthreads();
   const int nu = misc[0];
   int* rec_r = up.urec + size_t(r) * up.maxU * kUnitRecInts;
-  for (int x = tid; x < nu * n_anc; x += nt) {     // distinct records per (unit, slot)
+  // distinct records per (unit, slot): a warp per (unit, slot), a lane per position; the
+  // record of position j is new if j is the unit's first position or the slot changed there
+  const int nwarp = nt / 32;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int x = warp; x < nu * n_anc; x += nwarp) {
     const int k = x / n_anc, s = x % n_anc;
-    int cnt = 1;
-    for (int j = 1; j < un[k]; ++j) cnt += (fnew[ustart[k] + j] >> s) & 1;
-    sdist[k * TA + s] = cnt;
+    const bool in = lane < un[k];
+    const bool f = in && (lane == 0 || ((fnew[ustart[k] + lane] >> s) & 1));
+    const unsigned m = __ballot_sync(kFull, f);
+    if (lane == 0) sdist[k * TA + s] = __popc(m);
   }
   __syncthreads();
-  for (int x = tid; x < nu * n_anc; x += nt) {     // record list and per-position indices
+  for (int x = warp; x < nu * n_anc; x += nwarp) {  // record list and per-position indices
     const int k = x / n_anc, s = x % n_anc;
     int base = 0;
     for (int s2 = 0; s2 < s; ++s2) base += sdist[k * TA + s2];
-    int* rk = rec_r + size_t(k) * kUnitRecInts;
-    int c = 0;
-    for (int j = 0; j < un[k]; ++j) {
-      const int pos = ustart[k] + j;
-      if (j == 0 || ((fnew[pos] >> s) & 1)) {
-        rk[36 + base + c] = (s << 16) | spch[pos * TA + s];
-        ++c;
-      }
-      up.upos[(size_t(r) * B + pos) * 16 + s] = uint8_t(base + c - 1);
-    }
+    const bool in = lane < un[k];
+    const int pos = ustart[k] + lane;
+    const bool f = in && (lane == 0 || ((fnew[pos] >> s) & 1));
+    const unsigned m = __ballot_sync(kFull, f);
+    const int c = __popc(m & lt) + (f ? 1 : 0);      // records up to and including this position
+    if (f) rec_r[size_t(k) * kUnitRecInts + 36 + base + c - 1] = (s << 16) | spch[pos * TA + s];
+    if (in) up.upos[(size_t(r) * B + pos) * 16 + s] = uint8_t(base + c - 1);
   }
   for (int k = tid; k < nu; k += nt) {
     int* rk = rec_r + size_t(k) * kUnitRecInts;
