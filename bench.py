@@ -458,6 +458,126 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- operator sweep
+
+SWEEP_GEOMETRIES = tuple((dk, dv) for dk in (64, 128, 256) for dv in (64, 128, 256))
+SWEEP_REQUESTS = (1, 2, 8, 32, 64)
+SWEEP_BEAMS = (64, 256, 512)
+SWEEP_STEPS = (2, 4, 8)
+SWEEP_FULLSTATE_LIMIT = 96 << 30      # bytes of FullState ping-pong state the sweep allocates
+
+
+def fullstate_bytes_per_step(w: wl.Workload, parents: np.ndarray) -> list:
+    """Compulsory HBM bytes of each FullState step: every distinct parent's state read once
+    (step 1: the shared state), every beam's state written (fp32 d_v x d_k each), plus the
+    step inputs and o."""
+    e = w.elem_bytes
+    state = 4 * w.d_v * w.d_k
+    per_beam = state + (2 * w.d_k + w.d_v) * e + 8 + 4 * w.d_v
+    out = []
+    for t in range(w.T):
+        n_par = 1 if t == 0 else sum(len(np.unique(parents[t, r])) for r in range(w.R)) / w.R
+        out.append(int(w.R * w.H * (w.B * per_beam + n_par * state)))
+    return out
+
+
+def run_sweep(args):
+    """The operator sweep: nine (d_k, d_v) geometries x request counts x beam widths x decode
+    lengths (405 shapes), H = 16 heads, bf16 inputs, Zipf(1.0) parents, a shared state from a
+    1K-token prompt. Per shape: replay (tensor path) and FullState time per decode, capacity
+    bytes, algorithmic DRAM bytes and the fraction of the measured HBM bandwidth, and the
+    largest |o| difference between the two paths. One JSON line per shape."""
+    import torch
+    import linear_attention_beam_gdn_b200 as ola
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = measured_peaks()
+    geoms = SWEEP_GEOMETRIES if not args.sweep_geometry else \
+        tuple(tuple(int(x) for x in g.split("x")) for g in args.sweep_geometry.split(","))
+    Rs = SWEEP_REQUESTS if not args.sweep_requests else \
+        tuple(int(x) for x in args.sweep_requests.split(","))
+    Bs = SWEEP_BEAMS if not args.sweep_beams else tuple(int(x) for x in args.sweep_beams.split(","))
+    Ts = SWEEP_STEPS if not args.sweep_steps else tuple(int(x) for x in args.sweep_steps.split(","))
+    stream = torch.cuda.current_stream()
+
+    def timed(dec, steps, par, outs, reps, warm):
+        def decode():
+            dec.reset()
+            for t in range(len(steps)):
+                s = steps[t]
+                dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], par[t], out=outs[t])
+        for _ in range(warm):
+            decode()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            decode()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if dec.error() != ola.OLA_OK:
+            raise RuntimeError(f"device error: {ola.ola_strerror(dec.error())}")
+        return a.elapsed_time(b) / max(reps, 1)
+
+    for dk, dv in geoms:
+        for R in Rs:
+            base = wl.Workload(f"sweep_dk{dk}_dv{dv}_R{R}", R=R, H=16, d_k=dk, d_v=dv, P=1024,
+                               B=max(Bs), T=max(Ts), parent_law="zipf", zipf_s=1.0, seed=1005)
+            prompt = wl.make_prompt(base, dev)
+            S = ola.prefill(prompt["k"], prompt["v"], prompt["g"], prompt["beta"])
+            del prompt
+            for B in Bs:
+                for T in Ts:
+                    w = base.scaled(name=f"sweep_dk{dk}_dv{dv}_R{R}_B{B}_T{T}", B=B, T=T)
+                    steps = [wl.make_step_inputs(w, t, dev) for t in range(T)]
+                    parents = wl.make_parents(w)
+                    par = [torch.from_numpy(parents[t]).to(dev) for t in range(T)]
+                    outs = [torch.empty((R, B, w.H, dv), device=dev) for _ in range(T)]
+                    row = {"d_k": dk, "d_v": dv, "R": R, "H": w.H, "B": B, "T": T}
+                    bh_steps = R * w.H * B * T
+                    dec = ola.Decoder(S, B=B, T_max=T, in_dtype=w.torch_dtype,
+                                      path=ola.OLA_PATH_REPLAY, math=ola.OLA_MATH_TENSOR)
+                    t1 = timed(dec, steps, par, outs, 1, args.sweep_warmup)
+                    reps = max(1, min(args.sweep_reps, int(200.0 / max(t1, 1e-3))))
+                    ms = timed(dec, steps, par, outs, reps, 0)
+                    dec.close()
+                    rb = sum(algorithmic_bytes_per_step(w, parents))
+                    row["replay"] = {"ms": ms, "beam_head_steps_per_s": bh_steps / (ms / 1e3),
+                                     "bytes": int(rb), "gbs": rb / (ms / 1e3) / 1e9,
+                                     "hbm_frac": rb / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+                    o_rep = [o.clone() for o in outs] if args.sweep_check else None
+                    fsb = 2 * R * w.H * B * dv * dk * 4
+                    row["capacity"] = {
+                        "replay_record_bytes_per_beam_head_step": 4 * dv + w.elem_bytes * dk + 4,
+                        "replay_shared_state_bytes_per_request_head": 4 * dv * dk,
+                        "fullstate_bytes_per_beam_head": 4 * dv * dk,
+                        "fullstate_pingpong_bytes": fsb}
+                    if fsb <= SWEEP_FULLSTATE_LIMIT and not args.sweep_no_fullstate:
+                        dec = ola.Decoder(S, B=B, T_max=T, in_dtype=w.torch_dtype,
+                                          path=ola.OLA_PATH_FULLSTATE, math=ola.OLA_MATH_FP32)
+                        t1 = timed(dec, steps, par, outs, 1, min(args.sweep_warmup, 1))
+                        reps = max(1, min(args.sweep_reps, int(200.0 / max(t1, 1e-3))))
+                        fms = timed(dec, steps, par, outs, reps, 0)
+                        dec.close()
+                        fb = sum(fullstate_bytes_per_step(w, parents))
+                        row["fullstate"] = {"ms": fms, "bytes": int(fb),
+                                            "gbs": fb / (fms / 1e3) / 1e9,
+                                            "hbm_frac": fb / (fms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                                            "replay_speedup": fms / ms}
+                        if o_rep is not None:
+                            row["max_abs_diff_replay_vs_fullstate"] = max(
+                                float((a - b).abs().max()) for a, b in zip(o_rep, outs))
+                    else:
+                        row["fullstate"] = {"skipped": f"{fsb / 2**30:.1f} GiB of ping-pong state"}
+                    print(json.dumps(row), flush=True)
+                    del steps, par, outs, o_rep
+                    torch.cuda.empty_cache()
+            del S
+            torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -471,7 +591,20 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--requests", type=int, default=0,
                     help="override the workload's request count (profiling a smaller case)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="run the operator sweep (one JSON line per shape) instead of the bench")
+    ap.add_argument("--sweep-geometry", default="", help="e.g. 128x128,256x64 (d_k x d_v)")
+    ap.add_argument("--sweep-requests", default="")
+    ap.add_argument("--sweep-beams", default="")
+    ap.add_argument("--sweep-steps", default="")
+    ap.add_argument("--sweep-reps", type=int, default=10)
+    ap.add_argument("--sweep-warmup", type=int, default=2)
+    ap.add_argument("--sweep-check", action="store_true",
+                    help="also report the largest |o| difference between replay and FullState")
+    ap.add_argument("--sweep-no-fullstate", action="store_true")
     args = ap.parse_args()
+    if args.sweep:
+        return run_sweep(args)
     if args.warmup < 3 and args.impl == "ours":
         print("warm-up raised to 3", file=sys.stderr)
         args.warmup = 3
