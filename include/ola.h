@@ -150,6 +150,22 @@ ola_status ola_get_ancestry(ola_handle h, int32_t* out, void* stream);
 /* Wait for the handle's queued work, then return its sticky device error (OLA_OK if none). */
 ola_status ola_get_error(ola_handle h);
 
+/* Record reclamation ("Scientific Impact Assessment: OneLA", §1: append-only transition
+ * records over one shared post-prefill state, pruning through the parent-pointer ancestry
+ * index). Finds the longest prefix of chain slots at which every live beam of every request
+ * holds the same record (beam search that has converged), folds those records into S_ctx in
+ * chain order (S <- alpha_j S + w_j k_j^T, the transition written with the record; fp32, and
+ * the bf16 split of the tensor path is recomputed), moves the later records, chain rows and
+ * ranks down by that many slots and decreases t by it. Later steps give the same outputs up to
+ * rounding, and a decode can run past T_max while its beams keep converging. The current
+ * step's own records are never folded (t stays >= 1). ola_get_ancestry afterwards returns the
+ * chains without the folded slots, and ola_reset keeps the folded S_ctx.
+ *   out_folded : host int32, optional (NULL): number of folded steps (0 if none).
+ * Synchronises `stream`, which must be the stream of the handle's previous calls (or ordered
+ * after them). FullState handles hold no records: nothing is folded.
+ * Errors: INVALID_ARG (NULL handle), the sticky device error, CUDA. */
+ola_status ola_compact(ola_handle h, int32_t* out_folded, void* stream);
+
 /* Free every buffer of the handle (waits for its queued work first). NULL is a no-op.
  * The handle must not be used afterwards. */
 ola_status ola_destroy(ola_handle h);

@@ -67,6 +67,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "ola_current_step": (i32, [_P]),
         "ola_get_ancestry": (i32, [_P, _P, _P]),
         "ola_get_error": (i32, [_P]),
+        "ola_compact": (i32, [_P, ctypes.POINTER(ctypes.c_int32), _P]),
         "ola_destroy": (i32, [_P]),
         "ola_prefill": (i32, [i32, i32, i32, i32, i32, i32, _P, _P, _P, _P, _P, _P]),
         "ola_noalloc_scratch_bytes": (ctypes.c_uint64, [ctypes.POINTER(Geometry)]),
@@ -155,6 +156,13 @@ def ola_get_error(h) -> int:
 
 def ola_destroy(h) -> int:
     return lib().ola_destroy(h)
+
+
+def ola_compact(h, stream) -> tuple:
+    """(status, number of folded steps)."""
+    n = ctypes.c_int32(0)
+    st = lib().ola_compact(h, ctypes.byref(n), stream)
+    return st, n.value
 
 
 def ola_prefill(R, H, d_k, d_v, P, in_dtype, k, v, g, beta, S_out, stream) -> int:
@@ -305,6 +313,13 @@ class Decoder:
 
     def error(self) -> int:
         return ola_get_error(self.handle)
+
+    def compact(self, stream=None) -> int:
+        """Fold the chain steps every live beam shares into S_ctx and free their slots
+        (ola_compact); returns the number of folded steps."""
+        st, n = ola_compact(self.handle, _stream_ptr(stream))
+        _check(st, "ola_compact")
+        return n
 
     def reset(self) -> None:
         _check(ola_reset(self.handle), "ola_reset")

@@ -5,6 +5,9 @@
 
 #include <new>
 
+#include <algorithm>
+#include <vector>
+
 #include "ola_device.cuh"
 
 namespace ola {
@@ -36,6 +39,12 @@ bool make_record_maps(CUtensorMap* mkr, CUtensorMap* mw, const void* Kr, const v
                       uint64_t n_rec, int d_k, int d_v);
 cudaError_t launch_split_state(const float* S, void* hi, void* lo, int RH, int d_k, int d_v,
                                cudaStream_t stream);
+cudaError_t launch_common_prefix(const int* C, int R, int B, int T_max, int t, int* out,
+                                 cudaStream_t stream);
+cudaError_t launch_fold(float* S, const void* W, const void* Kr, int k_is_bf16, const float* A,
+                        const int* C, int R, int H, int d_k, int d_v, int B, int T_max, int t,
+                        int c, int layout, cudaStream_t stream);
+cudaError_t launch_chain_shift(int* C, int R, int B, int T_max, int t, int c, cudaStream_t stream);
 }  // namespace ola
 
 using namespace ola;
@@ -373,6 +382,60 @@ ola_status ola_reset(ola_handle h) {
   if (e != cudaSuccess) return from_cuda(e);
   h->t = 0;
   h->sticky = 0;
+  return OLA_OK;
+}
+
+ola_status ola_compact(ola_handle h, int32_t* out_folded, void* stream) {
+  if (!h) return OLA_ERR_INVALID_ARG;
+  if (out_folded) *out_folded = 0;
+  if (h->sticky) return static_cast<ola_status>(h->sticky);
+  const ola_geometry& g = h->g;
+  const int t = h->t;
+  if (g.path == OLA_PATH_FULLSTATE || t < 2) return OLA_OK;   // nothing to fold
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  // shared chain prefix of every request
+  int* lens = nullptr;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&lens), size_t(g.R) * 4, st);
+  if (e == cudaSuccess) e = launch_common_prefix(h->C, g.R, g.B, g.T_max, t, lens, st);
+  std::vector<int> host(size_t(g.R), 0);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(host.data(), lens, size_t(g.R) * 4, cudaMemcpyDeviceToHost, st);
+  if (lens) cudaFreeAsync(lens, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return from_cuda(e);
+  int c = t - 1;
+  for (int x : host) c = std::min(c, x);
+  if (c <= 0) return OLA_OK;
+  // fold the shared records into S_ctx (and its bf16 split), then move the later record slots
+  // and the chain rows down by c
+  const int layout = h->mma ? 1 : 0;
+  e = launch_fold(h->S, h->W, h->Kr, g.in_dtype == OLA_BF16, h->A, h->C, g.R, g.H, g.d_k, g.d_v,
+                  g.B, g.T_max, t, c, layout, st);
+  if (e == cudaSuccess && g.math == OLA_MATH_TENSOR)
+    e = launch_split_state(h->S, h->S_hi, h->S_lo, g.R * g.H, g.d_k, g.d_v, st);
+  const size_t rows = size_t(g.R) * g.H * g.B;
+  const size_t kbytes = g.in_dtype == OLA_BF16 ? 2 : 4;
+  const size_t w_slot = rows * g.d_v * 4, k_slot = rows * g.d_k * kbytes, a_slot = rows * 4;
+  for (int s = c; s < t && e == cudaSuccess; ++s) {   // increasing order: sources stay intact
+    char* W = reinterpret_cast<char*>(h->W);
+    char* K = static_cast<char*>(h->Kr);
+    char* A = reinterpret_cast<char*>(h->A);
+    e = cudaMemcpyAsync(W + (s - c) * w_slot, W + s * w_slot, w_slot, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(K + (s - c) * k_slot, K + s * k_slot, k_slot, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(A + (s - c) * a_slot, A + s * a_slot, a_slot, cudaMemcpyDeviceToDevice, st);
+  }
+  if (e == cudaSuccess) e = launch_chain_shift(h->C, g.R, g.B, g.T_max, t, c, st);
+  // the next step reads the depth-first ranks of this one from the buffer of its parity
+  const size_t RB = size_t(g.R) * g.B;
+  if (e == cudaSuccess && h->rank && (c & 1))
+    e = cudaMemcpyAsync(h->rank + size_t((t - c) & 1) * RB, h->rank + size_t(t & 1) * RB, RB * 4,
+                        cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  h->t = t - c;
+  if (out_folded) *out_folded = c;
   return OLA_OK;
 }
 

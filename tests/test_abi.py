@@ -101,6 +101,7 @@ def test_null_arguments(L):
     assert L.ola_current_step(None) == -1
     assert L.ola_step(None, 16, 16, 16, 16, 16, 16, 16, None) == ola.OLA_ERR_INVALID_ARG
     assert L.ola_get_ancestry(None, 16, None) == ola.OLA_ERR_INVALID_ARG
+    assert L.ola_compact(None, None, None) == ola.OLA_ERR_INVALID_ARG
 
 
 def test_prefill_validation(L):

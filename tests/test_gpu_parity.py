@@ -256,3 +256,73 @@ def test_shape_checks_in_binding():
         with pytest.raises(TypeError):
             dec.step(s["q"].float(), s["k"], s["v"], s["g"], s["beta"],
                      torch.zeros((w.R, w.B), dtype=torch.int32, device="cuda"))
+
+
+# ----------------------------------------------------------------------------- reclamation
+
+def _converging_parents(w, merge_steps):
+    """Zipf parents, except that at each step in `merge_steps` (0-based) every new beam takes
+    beam 0 as its parent: after such a step all chains share every earlier slot."""
+    par = wl.make_parents(w)
+    for t in merge_steps:
+        par[t] = 0
+    return par
+
+
+@pytest.mark.parametrize("path", ["replay_tensor", "replay_fp32"])
+def test_compact_decodes_past_t_max(path):
+    """A decode of 8 steps on a handle of T_max = 4: ola_compact after steps 3 and 6 folds the
+    chain slots every beam shares into S_ctx, and the outputs of every step still match the
+    oracle's full-state decode (which has no capacity limit); the ancestry after the last step
+    equals the oracle's chains without the folded slots."""
+    w = wl.WORKLOADS["single_request"].scaled(H=2, B=40, P=64, T=8)
+    S32, steps, dev_steps, _ = small_problem(w)
+    parents = _converging_parents(w, merge_steps=[2, 5])
+    ref = oracle_outputs(S32, steps, parents)
+    p, m = PATHS[path]
+    dev = torch.device("cuda")
+    dec = ola.Decoder(S32.cuda(), B=w.B, T_max=4, in_dtype=w.torch_dtype, path=p, math=m)
+    folded, outs = [], []
+    try:
+        for t in range(w.T):
+            s = dev_steps[t]
+            par = torch.from_numpy(parents[t]).to(dev)
+            outs.append(dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], par).cpu())
+            if t in (2, 5):
+                folded.append(dec.compact())
+        anc = dec.ancestry().cpu().numpy()
+        assert dec.error() == ola.OLA_OK
+        # after step 3 (1-based) every chain shares slots 0..1; after step 6 slots 0..2 of the
+        # compacted chains (steps 3..5)
+        assert folded == [2, 3]
+        assert dec.t == 8 - 5
+    finally:
+        dec.close()
+    o = torch.stack(outs).double().numpy()
+    err = max_abs(o, ref)
+    assert err <= tol_for(path), (path, err)
+    assert np.array_equal(anc, oracle.ancestry_table(parents)[:, :, 5:])
+
+
+def test_compact_without_shared_prefix_changes_nothing():
+    """With no chain slot shared by every beam nothing is folded, and the next steps match the
+    oracle as without the call."""
+    w = wl.WORKLOADS["single_request"].scaled(H=2, B=40, P=64, T=4)
+    S32, steps, dev_steps, parents = small_problem(w)
+    assert len(np.unique(parents[1, 0])) > 1        # step 2 keeps several parents
+    ref = oracle_outputs(S32, steps, parents)
+    dev = torch.device("cuda")
+    dec = ola.Decoder(S32.cuda(), B=w.B, T_max=4, in_dtype=w.torch_dtype,
+                      path=ola.OLA_PATH_REPLAY, math=ola.OLA_MATH_TENSOR)
+    outs = []
+    try:
+        for t in range(w.T):
+            s = dev_steps[t]
+            outs.append(dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"],
+                                 torch.from_numpy(parents[t]).to(dev)).cpu())
+            if t == 1:
+                assert dec.compact() == 0
+        assert dec.error() == ola.OLA_OK
+    finally:
+        dec.close()
+    assert max_abs(torch.stack(outs).double().numpy(), ref) <= tol_for("replay_tensor")
