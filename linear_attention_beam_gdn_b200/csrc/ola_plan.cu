@@ -88,9 +88,11 @@ size_t plan_units_smem(int B, int T_max) {
   const int Bp = (B + 3) & ~3, TA = T_max > 1 ? T_max - 1 : 1;
   // keys, parents, perm, chains, change masks, unit of position, unit start/size/U, counts,
   // sibling-group starts and sizes, prefix sums of group sizes and new-record counts, unit
-  // ends, scratch
+  // ends, per-chunk key counts of the sort (16 x B uint16), per-position record indices
+  // (B x 16 bytes), scratch
   return sizeof(int) * (size_t(Bp) + B + B + size_t(B) * TA + B + B + 3 * size_t(B) +
-                        size_t(B) * TA + 2 * size_t(B) + 3 * size_t(B + 1) + 128);
+                        size_t(B) * TA + 2 * size_t(B) + 3 * size_t(B + 1) + 8 * size_t(B) +
+                        4 * size_t(B) + 4 + 128);
 }
 
 __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up) {
@@ -113,7 +115,11 @@ __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up
   int* PS = gsz + B;              // [B + 1] prefix sums of the group sizes
   int* PC = PS + (B + 1);         // [B + 1] prefix sums of the groups' new-record counts
   int* gnext = PC + (B + 1);      // [B + 1] end (exclusive) of a unit starting at group g
-  int* misc = gnext + (B + 1);    // [0] unit count, [1] last-CTA flag, [2] groups, [32..] scratch
+  unsigned short* ccnt = reinterpret_cast<unsigned short*>(gnext + (B + 1));   // [16][B]
+  int* upos_i = gnext + (B + 1) + 8 * B;
+  upos_i += (4 - (reinterpret_cast<uintptr_t>(upos_i) >> 2) % 4) % 4;           // 16-byte aligned
+  uint8_t* upos_s = reinterpret_cast<uint8_t*>(upos_i);                        // [B][16]
+  int* misc = upos_i + 4 * B;     // [0] unit count, [1] last-CTA flag, [2] groups, [32..] scratch
 
   // depth-first order: stable sort of the beams by their parent's position (ola_plan.cu above)
   for (int b = tid; b < Bp; b += nt) {
@@ -126,21 +132,69 @@ __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up
     keys[b] = key;
   }
   __syncthreads();
-  const int4* k4 = reinterpret_cast<const int4*>(keys);
-  for (int b = tid; b < B; b += nt) {
-    const int k = keys[b];
-    int pos = 0;
-    for (int j = 0; j < Bp / 4; ++j) {
-      const int4 kk = k4[j];
-      const int b2 = 4 * j;
-      pos += (kk.x < k) | ((kk.x == k) & (b2 + 0 < b));
-      pos += (kk.y < k) | ((kk.y == k) & (b2 + 1 < b));
-      pos += (kk.z < k) | ((kk.z == k) & (b2 + 2 < b));
-      pos += (kk.w < k) | ((kk.w == k) & (b2 + 3 < b));
+  if (B <= 512 && nt == 512) {
+    // counting sort, stable: a warp per chunk of 32 beams finds the beams of its chunk with
+    // equal keys (match), per key the counts of the earlier chunks are summed, and the key
+    // offsets come from a scan; position = beams with a smaller key + beams with the same key
+    // in earlier chunks + those earlier in this chunk
+    int* off = ustart;                              // [B] (free until the unit cut)
+    for (int x = tid; x < 16 * B; x += nt) ccnt[x] = 0;
+    __syncthreads();
+    const int b = 32 * warp + lane;
+    const bool valid = b < B;
+    const int k = valid ? keys[b] : -1 - lane;
+    const unsigned peers = __match_any_sync(kFull, k);
+    const int rin = __popc(peers & ((1u << lane) - 1u));
+    if (valid && lane == __ffs(peers) - 1) ccnt[warp * B + k] = (unsigned short)__popc(peers);
+    __syncthreads();
+    for (int kk = tid; kk < B; kk += nt) {
+      int run = 0;
+      for (int j = 0; j < 16; ++j) {
+        const int c = ccnt[j * B + kk];
+        ccnt[j * B + kk] = (unsigned short)run;
+        run += c;
+      }
+      off[kk] = run;                                // beams with key kk
     }
-    a.perm[size_t(r) * B + pos] = b;
-    a.rank_cur[size_t(r) * B + b] = pos;
-    sperm[pos] = b;
+    __syncthreads();
+    {                                               // exclusive scan of off over the keys
+      const int v = tid < B ? off[tid] : 0;
+      int x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) misc[32 + warp] = x;
+      __syncthreads();
+      int before = 0;
+      for (int w2 = 0; w2 < warp; ++w2) before += misc[32 + w2];
+      if (tid < B) off[tid] = before + x - v;
+      __syncthreads();
+    }
+    if (valid) {
+      const int pos = off[k] + ccnt[warp * B + k] + rin;
+      a.perm[size_t(r) * B + pos] = b;
+      a.rank_cur[size_t(r) * B + b] = pos;
+      sperm[pos] = b;
+    }
+  } else {
+    const int4* k4 = reinterpret_cast<const int4*>(keys);
+    for (int b = tid; b < B; b += nt) {
+      const int k = keys[b];
+      int pos = 0;
+      for (int j = 0; j < Bp / 4; ++j) {
+        const int4 kk = k4[j];
+        const int b2 = 4 * j;
+        pos += (kk.x < k) | ((kk.x == k) & (b2 + 0 < b));
+        pos += (kk.y < k) | ((kk.y == k) & (b2 + 1 < b));
+        pos += (kk.z < k) | ((kk.z == k) & (b2 + 2 < b));
+        pos += (kk.w < k) | ((kk.w == k) & (b2 + 3 < b));
+      }
+      a.perm[size_t(r) * B + pos] = b;
+      a.rank_cur[size_t(r) * B + b] = pos;
+      sperm[pos] = b;
+    }
   }
   __syncthreads();
   // parent chains by position; chain rows of the new beams (a thread per position: the parent's
@@ -318,7 +372,13 @@ __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up
     const unsigned m = __ballot_sync(kFull, f);
     const int c = __popc(m & lt) + (f ? 1 : 0);      // records up to and including this position
     if (f) rec_r[size_t(k) * kUnitRecInts + 36 + base + c - 1] = (s << 16) | spch[pos * TA + s];
-    if (in) up.upos[(size_t(r) * B + pos) * 16 + s] = uint8_t(base + c - 1);
+    if (in) upos_s[pos * 16 + s] = uint8_t(base + c - 1);
+  }
+  __syncthreads();
+  {                                                 // per-position record indices, 16 B a row
+    const uint4* src = reinterpret_cast<const uint4*>(upos_s);
+    uint4* dst = reinterpret_cast<uint4*>(up.upos + size_t(r) * B * 16);
+    for (int pos = tid; pos < B; pos += nt) dst[pos] = src[pos];
   }
   for (int k = tid; k < nu; k += nt) {
     int* rk = rec_r + size_t(k) * kUnitRecInts;
