@@ -362,10 +362,18 @@ __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up
     if (lane == 0) sdist[k * TA + s] = __popc(m);
   }
   __syncthreads();
+  for (int k = tid; k < nu; k += nt) {              // counts -> offsets of each slot's records
+    int run = 0;
+    for (int s = 0; s < n_anc; ++s) {
+      const int c = sdist[k * TA + s];
+      sdist[k * TA + s] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
   for (int x = warp; x < nu * n_anc; x += nwarp) {  // record list and per-position indices
     const int k = x / n_anc, s = x % n_anc;
-    int base = 0;
-    for (int s2 = 0; s2 < s; ++s2) base += sdist[k * TA + s2];
+    const int base = sdist[k * TA + s];
     const bool in = lane < un[k];
     const int pos = ustart[k] + lane;
     const bool f = in && (lane == 0 || ((fnew[pos] >> s) & 1));
