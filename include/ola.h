@@ -134,6 +134,21 @@ ola_status ola_step_host(ola_handle h, const void* q, const void* k, const void*
                          const float* g, const float* beta, const int32_t* parent_idx,
                          float* out_o, void* stream);
 
+/* ola_step_host without waiting: pipelined decode from host buffers. The inputs are copied
+ * in on a copy stream of the handle, the step runs on `stream` and out_o is copied back on a
+ * second copy stream, so one call's copy-out overlaps the next call's copy-in (the host link
+ * carries both directions at once). Two device staging sets are used in turn. Returns once the
+ * work is queued. The host buffers of a call must stay valid, and out_o unread, until
+ * ola_host_sync; they must be pinned for the copies to be asynchronous.
+ * Errors: as ola_step; INVALID_ARG for NULL pointers; CUDA. */
+ola_status ola_step_host_async(ola_handle h, const void* q, const void* k, const void* v,
+                               const float* g, const float* beta, const int32_t* parent_idx,
+                               float* out_o, void* stream);
+
+/* Wait for every queued ola_step_host_async call (its copies and steps); then as
+ * ola_get_error. */
+ola_status ola_host_sync(ola_handle h);
+
 /* Rewind to t = 0, keeping S_ctx, and clear the sticky device error. Stream-ordered on the
  * stream of the handle's last call (no host synchronisation): work queued before it still
  * runs, and the next ola_step must be queued on that stream or ordered after it. */

@@ -63,6 +63,8 @@ def _declare(L: ctypes.CDLL) -> None:
         "ola_create": (i32, [ctypes.POINTER(Geometry), _P, _P, ctypes.POINTER(_P)]),
         "ola_step": (i32, [_P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "ola_step_host": (i32, [_P, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "ola_step_host_async": (i32, [_P, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "ola_host_sync": (i32, [_P]),
         "ola_reset": (i32, [_P]),
         "ola_current_step": (i32, [_P]),
         "ola_get_ancestry": (i32, [_P, _P, _P]),
@@ -136,6 +138,14 @@ def ola_step(h, q, k, v, g, beta, parent_idx, out_o, stream) -> int:
 
 def ola_step_host(h, q, k, v, g, beta, parent_idx, out_o, stream) -> int:
     return lib().ola_step_host(h, q, k, v, g, beta, parent_idx, out_o, stream)
+
+
+def ola_step_host_async(h, q, k, v, g, beta, parent_idx, out_o, stream) -> int:
+    return lib().ola_step_host_async(h, q, k, v, g, beta, parent_idx, out_o, stream)
+
+
+def ola_host_sync(h) -> int:
+    return lib().ola_host_sync(h)
 
 
 def ola_reset(h) -> int:
@@ -301,6 +311,25 @@ class Decoder:
                 _need(out, (R, B, H, dv), torch.float32, "out_o", cpu)]
         _check(ola_step_host(self.handle, *ptrs, _stream_ptr(stream)), "ola_step_host")
         return out
+
+    def step_host_async(self, q, k, v, g, beta, parent_idx, out, stream=None):
+        """ola_step_host_async: CPU tensors (pinned); `out` is complete after host_sync()."""
+        torch = _torch()
+        cpu = torch.device("cpu")
+        R, B, H, dk, dv = self.R, self.B, self.H, self.d_k, self.d_v
+        dt = self.in_dtype
+        ptrs = [_need(q, (R, B, H, dk), dt, "q", cpu), _need(k, (R, B, H, dk), dt, "k", cpu),
+                _need(v, (R, B, H, dv), dt, "v", cpu),
+                _need(g, (R, B, H), torch.float32, "g", cpu),
+                _need(beta, (R, B, H), torch.float32, "beta", cpu),
+                _need(parent_idx, (R, B), torch.int32, "parent_idx", cpu),
+                _need(out, (R, B, H, dv), torch.float32, "out_o", cpu)]
+        _check(ola_step_host_async(self.handle, *ptrs, _stream_ptr(stream)),
+               "ola_step_host_async")
+        return out
+
+    def host_sync(self) -> None:
+        _check(ola_host_sync(self.handle), "ola_host_sync")
 
     def ancestry(self, stream=None):
         """Chains of the current beams: [R, B, t] int32 (device)."""

@@ -75,6 +75,14 @@ struct ola_ctx {
   // staging buffers of ola_step_host (allocated on first use)
   void* st[7] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
   cudaStream_t last_stream = nullptr;
+  // pipelined host-buffer steps (ola_step_host_async): two staging sets used alternately, a
+  // copy-in and a copy-out stream, and the events that order them with the compute stream
+  struct {
+    void* buf[2][7] = {};
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+    long long n = 0;                 // calls so far
+  } hp;
 };
 
 namespace {
@@ -166,6 +174,16 @@ void free_all(ola_ctx* h) {
     if (p) cudaFree(p);
   for (void* p : h->st)
     if (p) cudaFree(p);
+  for (auto& set : h->hp.buf)
+    for (void* p : set)
+      if (p) cudaFree(p);
+  for (int i = 0; i < 2; ++i) {
+    if (h->hp.in_done[i]) cudaEventDestroy(h->hp.in_done[i]);
+    if (h->hp.comp_done[i]) cudaEventDestroy(h->hp.comp_done[i]);
+    if (h->hp.out_done[i]) cudaEventDestroy(h->hp.out_done[i]);
+  }
+  if (h->hp.s_in) cudaStreamDestroy(h->hp.s_in);
+  if (h->hp.s_out) cudaStreamDestroy(h->hp.s_out);
 }
 
 StepArgs make_args(ola_ctx* h, const void* q, const void* k, const void* v, const float* g,
@@ -376,6 +394,68 @@ ola_status ola_step_host(ola_handle h, const void* q, const void* k, const void*
   return from_cuda(cudaStreamSynchronize(st));
 }
 
+ola_status ola_step_host_async(ola_handle h, const void* q, const void* k, const void* v,
+                               const float* g, const float* beta, const int32_t* parent_idx,
+                               float* out_o, void* stream) {
+  if (!h) return OLA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !g || !beta || !parent_idx || !out_o) return OLA_ERR_INVALID_ARG;
+  auto& hp = h->hp;
+  const size_t R = h->g.R, B = h->g.B, H = h->g.H;
+  const size_t e = h->g.in_dtype == OLA_BF16 ? 2 : 4;
+  const size_t bytes[7] = {R * B * H * h->g.d_k * e, R * B * H * h->g.d_k * e,
+                           R * B * H * h->g.d_v * e, R * B * H * 4, R * B * H * 4, R * B * 4,
+                           R * B * H * h->g.d_v * 4};
+  cudaError_t ce = cudaSuccess;
+  if (!hp.s_in) {
+    ce = cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking);
+    if (ce == cudaSuccess) ce = cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking);
+    for (int i = 0; i < 2 && ce == cudaSuccess; ++i) {
+      ce = cudaEventCreateWithFlags(&hp.in_done[i], cudaEventDisableTiming);
+      if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming);
+      if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming);
+      for (int j = 0; j < 7 && ce == cudaSuccess; ++j) ce = cudaMalloc(&hp.buf[i][j], bytes[j]);
+    }
+    if (ce != cudaSuccess) return from_cuda(ce);
+  }
+  const int p = int(hp.n & 1);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // copy-in: staging set p is free once the step of two calls ago has run
+  if (hp.n >= 2) ce = cudaStreamWaitEvent(hp.s_in, hp.comp_done[p], 0);
+  const void* src[6] = {q, k, v, g, beta, parent_idx};
+  for (int i = 0; i < 6 && ce == cudaSuccess; ++i)
+    ce = cudaMemcpyAsync(hp.buf[p][i], src[i], bytes[i], cudaMemcpyHostToDevice, hp.s_in);
+  if (ce == cudaSuccess) ce = cudaEventRecord(hp.in_done[p], hp.s_in);
+  // the step, on the caller's stream, after its inputs and after o of two calls ago is out
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, hp.in_done[p], 0);
+  if (ce == cudaSuccess && hp.n >= 2) ce = cudaStreamWaitEvent(cs, hp.out_done[p], 0);
+  if (ce != cudaSuccess) return from_cuda(ce);
+  ola_status s = ola_step(h, hp.buf[p][0], hp.buf[p][1], hp.buf[p][2],
+                          static_cast<const float*>(hp.buf[p][3]),
+                          static_cast<const float*>(hp.buf[p][4]),
+                          static_cast<const int32_t*>(hp.buf[p][5]),
+                          static_cast<float*>(hp.buf[p][6]), stream);
+  if (s != OLA_OK) return s;
+  // copy-out, overlapping the next call's copy-in (the link carries both directions at once)
+  ce = cudaEventRecord(hp.comp_done[p], cs);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(hp.s_out, hp.comp_done[p], 0);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpyAsync(out_o, hp.buf[p][6], bytes[6], cudaMemcpyDeviceToHost, hp.s_out);
+  if (ce == cudaSuccess) ce = cudaEventRecord(hp.out_done[p], hp.s_out);
+  if (ce != cudaSuccess) return from_cuda(ce);
+  ++hp.n;
+  return OLA_OK;
+}
+
+ola_status ola_host_sync(ola_handle h) {
+  if (!h) return OLA_ERR_INVALID_ARG;
+  if (h->hp.s_out) {
+    cudaError_t ce = cudaStreamSynchronize(h->hp.s_in);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(h->hp.s_out);
+    if (ce != cudaSuccess) return from_cuda(ce);
+  }
+  return ola_get_error(h);
+}
+
 ola_status ola_reset(ola_handle h) {
   if (!h) return OLA_ERR_INVALID_ARG;
   cudaError_t e = cudaMemsetAsync(h->err, 0, 16, h->last_stream);
@@ -464,6 +544,10 @@ ola_status ola_get_error(ola_handle h) {
 ola_status ola_destroy(ola_handle h) {
   if (!h) return OLA_OK;
   cudaStreamSynchronize(h->last_stream);
+  if (h->hp.s_out) {
+    cudaStreamSynchronize(h->hp.s_in);
+    cudaStreamSynchronize(h->hp.s_out);
+  }
   free_all(h);
   delete h;
   return OLA_OK;

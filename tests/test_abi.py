@@ -102,6 +102,9 @@ def test_null_arguments(L):
     assert L.ola_step(None, 16, 16, 16, 16, 16, 16, 16, None) == ola.OLA_ERR_INVALID_ARG
     assert L.ola_get_ancestry(None, 16, None) == ola.OLA_ERR_INVALID_ARG
     assert L.ola_compact(None, None, None) == ola.OLA_ERR_INVALID_ARG
+    assert L.ola_step_host_async(None, 16, 16, 16, 16, 16, 16, 16, None) == \
+        ola.OLA_ERR_INVALID_ARG
+    assert L.ola_host_sync(None) == ola.OLA_ERR_INVALID_ARG
 
 
 def test_prefill_validation(L):

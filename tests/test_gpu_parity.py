@@ -190,6 +190,31 @@ def test_step_host_matches_step():
         dec.close()
 
 
+def test_step_host_async_matches_step():
+    """The pipelined host-buffer entry point (two staging sets, copy-in and copy-out streams)
+    gives the device path's outputs bit for bit, over two decodes and more steps than staging
+    sets."""
+    w = wl.WORKLOADS["single_request"].scaled(H=2, P=32, T=5)
+    S32, steps, dev_steps, parents = small_problem(w)
+    o_dev, _, _ = run_library(S32.cuda(), dev_steps, parents, "replay_tensor", w.torch_dtype)
+    dec = ola.Decoder(S32.cuda(), B=w.B, T_max=w.T, in_dtype=w.torch_dtype)
+    hs = [{k: v.pin_memory() for k, v in steps[t].items()} for t in range(w.T)]
+    hp = [torch.from_numpy(parents[t]).pin_memory() for t in range(w.T)]
+    try:
+        for _ in range(2):
+            dec.reset()
+            outs = [torch.full((w.R, w.B, w.H, w.d_v), float("nan")).pin_memory()
+                    for _ in range(w.T)]
+            for t in range(w.T):
+                s = hs[t]
+                dec.step_host_async(s["q"], s["k"], s["v"], s["g"], s["beta"], hp[t], outs[t])
+            dec.host_sync()
+            for t in range(w.T):
+                assert np.array_equal(outs[t].double().numpy(), o_dev[t]), t
+    finally:
+        dec.close()
+
+
 # ----------------------------------------------------------------------------- errors
 
 def test_bad_parent_is_sticky_and_reset_clears():
