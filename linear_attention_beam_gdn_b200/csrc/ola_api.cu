@@ -14,6 +14,10 @@ namespace ola {
 cudaError_t launch_prefill(int R, int H, int d_k, int d_v, int P, int in_dtype, const void* k,
                            const void* v, const float* g, const float* beta, float* S_out,
                            cudaStream_t stream);
+bool prefill_chunk_supported(int d_k, int d_v, int in_dtype, const void* k, const void* v);
+cudaError_t launch_prefill_chunk(int R, int H, int P, const void* k, const void* v,
+                                 const float* g, const float* beta, float* S_out, int* err,
+                                 cudaStream_t stream);
 cudaError_t launch_fullstate(const StepArgs& a, int in_dtype, cudaStream_t stream);
 cudaError_t launch_replay_simt(const StepArgs& a, int in_dtype, cudaStream_t stream);
 size_t replay_simt_smem(int d_k, int d_v, int T_max);
@@ -561,8 +565,24 @@ ola_status ola_prefill(int32_t R, int32_t H, int32_t d_k, int32_t d_v, int32_t P
   if (!pow2_width(d_k) || !pow2_width(d_v)) return OLA_ERR_UNSUPPORTED;
   if (!S_out || !aligned(S_out, 16)) return OLA_ERR_INVALID_ARG;
   if (P > 0 && (!k || !v || !g || !beta)) return OLA_ERR_INVALID_ARG;
-  return from_cuda(launch_prefill(R, H, d_k, d_v, P, in_dtype, k, v, g, beta, S_out,
-                                  static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (P > 0 && prefill_chunk_supported(d_k, d_v, in_dtype, k, v)) {
+    // chunked tensor-core form; waits for it so that a device-side timeout is returned
+    int* derr = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&derr), 4 * sizeof(int), st) != cudaSuccess)
+      return OLA_ERR_OOM;
+    int herr[4] = {0, 0, 0, 0};
+    cudaError_t e = cudaMemsetAsync(derr, 0, 4 * sizeof(int), st);
+    if (e == cudaSuccess) e = launch_prefill_chunk(R, H, P, k, v, g, beta, S_out, derr, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(herr, derr, sizeof(herr), cudaMemcpyDeviceToHost, st);
+    const cudaError_t ef = cudaFreeAsync(derr, st);
+    if (e == cudaSuccess) e = ef;
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return from_cuda(e);
+    return herr[0] != 0 ? static_cast<ola_status>(herr[0]) : OLA_OK;
+  }
+  return from_cuda(launch_prefill(R, H, d_k, d_v, P, in_dtype, k, v, g, beta, S_out, st));
 }
 
 }  // extern "C"

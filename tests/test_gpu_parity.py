@@ -51,6 +51,48 @@ def test_prefill_matches_oracle(name):
     assert err <= 1e-4
 
 
+@pytest.mark.parametrize("P", [1, 63, 64, 65, 1000])
+def test_prefill_chunked_ragged_lengths(P):
+    """d_k = d_v = 128 with a bf16 prompt runs the chunked tensor-core prefill (64 tokens per
+    chunk): prompts that end inside, at and just past a chunk boundary, and one of many chunks
+    with a ragged tail, against the fp64 token recurrence."""
+    w = wl.WORKLOADS["single_request"].scaled(R=2, H=3, P=P)
+    prompt = wl.make_prompt(w, "cpu")
+    S_ref = oracle_prefill_all(prompt)
+    dp = {k: v.cuda() for k, v in prompt.items()}
+    S = ola.prefill(dp["k"], dp["v"], dp["g"], dp["beta"])
+    assert bool(torch.isfinite(S).all())
+    err = max_abs(S.double().cpu().numpy(), S_ref)
+    print(f"chunked prefill P={P}: max-abs {err:.3e}")
+    assert err <= 1e-4
+
+
+def test_prefill_chunked_weak_decay():
+    """alpha = exp(-0.01) on every token: the state keeps the contributions of all 32 chunks,
+    where the rounding of the bf16 hi/lo operands (relative 2^-17 per product) accumulates the
+    most instead of decaying away. Bound: 32 chunks x a few such roundings on entries of order 1,
+    well inside 2e-3."""
+    w = wl.WORKLOADS["single_request"].scaled(R=1, H=2, P=2048)
+    prompt = wl.make_prompt(w, "cpu")
+    prompt["g"] = torch.full_like(prompt["g"], -0.01)
+    S_ref = oracle_prefill_all(prompt)
+    dp = {k: v.cuda() for k, v in prompt.items()}
+    S = ola.prefill(dp["k"], dp["v"], dp["g"], dp["beta"])
+    assert bool(torch.isfinite(S).all())
+    err = max_abs(S.double().cpu().numpy(), S_ref)
+    print(f"chunked prefill, weak decay: max-abs {err:.3e}, max |S| {np.abs(S_ref).max():.2f}")
+    assert err <= 2e-3
+
+
+def test_prefill_chunked_repeated_call_is_deterministic():
+    """Same prompt twice: bit-identical states (fixed reduction order in every kernel)."""
+    w = wl.WORKLOADS["single_request"].scaled(R=1, H=4, P=300)
+    dp = {k: v.cuda() for k, v in wl.make_prompt(w, "cpu").items()}
+    S1 = ola.prefill(dp["k"], dp["v"], dp["g"], dp["beta"])
+    S2 = ola.prefill(dp["k"], dp["v"], dp["g"], dp["beta"])
+    assert torch.equal(S1, S2)
+
+
 def test_prefill_zero_tokens_gives_zero_state():
     w = wl.WORKLOADS["tiny"].scaled(P=0)
     k = torch.empty((1, 0, 2, 16), device="cuda")
