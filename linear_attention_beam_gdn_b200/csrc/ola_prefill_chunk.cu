@@ -16,7 +16,8 @@
 //
 // One CTA per (request, head), one per SM (tensor memory: 448 of 512 columns):
 //   warps 0-3  per chunk, one chunk ahead of the state chain: gates (prefix sums, a, D), L from
-//              K K^T, T by 16 x 16 block forward substitution in fp32, T as bf16 hi + lo tiles
+//              K K^T, T in fp32 by 16 x 16 blocks (diagonal blocks by forward substitution,
+//              then T_ba = -T_bb sum_{a <= c < b} L_bc T_ca by block distance), T as bf16 hi + lo
 //   warps 4-7  state rows (thread = row = tensor-memory lane): R, W D, and the state entering
 //              the next chunk (its bf16 hi + lo for Z, and a_C S for the accumulation)
 //   warp 8     TMA: key and value tiles of each chunk, three stages
@@ -52,19 +53,21 @@ constexpr uint32_t kTG = 384;      // K K^T, M = 64 layout (64 columns)
 constexpr uint32_t kTile = kC * kD * 2;                        // 16 KB: [2 col blocks][64][128 B]
 constexpr uint32_t kTTile = kC * kC * 2;                       // 8 KB: [64][64] bf16, sw128
 constexpr int kScFloats = 3 * kC + 4;                          // a, beta, D, a_C (+ pad)
-constexpr int kLd = kC + 1;                                    // padded fp32 row of L and T
+constexpr int kLd = kC + 1;                                    // padded fp32 row of L
+constexpr int kLdT = kC + 4;                                   // fp32 row of T (16-byte rows)
 constexpr uint32_t kOffK = 0;                                  // keys, 128-byte swizzle
 constexpr uint32_t kOffV = kOffK + kStages * kTile;            // values, no swizzle
 constexpr uint32_t kOffT = kOffV + kStages * kTile;            // T hi, T lo per stage
 constexpr uint32_t kOffSc = kOffT + kStages * 2 * kTTile;      // gate scalars per stage
 constexpr uint32_t kOffL = kOffSc + kStages * kScFloats * 4;   // L fp32 [64][65]
-constexpr uint32_t kOffTf = kOffL + kC * kLd * 4;              // T fp32 [64][65]
-constexpr uint32_t kOffQ = kOffTf + kC * kLd * 4;              // block products [3][16][16]
+constexpr uint32_t kOffTf = kOffL + kC * kLd * 4;              // T fp32 [64][68]
+constexpr uint32_t kOffQ = kOffTf + kC * kLdT * 4;             // block products [3][16][16]
 constexpr uint32_t kOffG = kOffQ + 3 * 256 * 4;                // G_j [64] + a warp total
 constexpr uint32_t kOffBar = kOffG + (kC + 4) * 4;
 constexpr int kNumBars = 18;
 constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + holder, alignment
 static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
+static_assert(kOffTf % 16 == 0 && kOffQ % 16 == 0, "float4 rows of T and of the block products");
 static_assert(kOffT % 1024 == 0 && kOffV % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
@@ -393,6 +396,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
     float* Tf = reinterpret_cast<float*>(sm + kOffTf);
     float* Qb = reinterpret_cast<float*>(sm + kOffQ);
     float* Gs = reinterpret_cast<float*>(sm + kOffG);
+    // gates of chunk c (tokens past P: g = 0, beta = 0, an identity step), loaded a chunk ahead
+    auto load_gates = [&](int c, float& gv, float& bv) {
+      gv = 0.f;
+      bv = 0.f;
+      const int p = kC * c + tid;
+      if (tid < kC && c < nch && p < a.P) {
+        const size_t ix = (size_t(r) * a.P + p) * a.H + h;
+        gv = __ldg(a.g + ix);
+        bv = __ldg(a.beta + ix);
+      }
+    };
+    float gj, bj;
+    load_gates(0, gj, bj);
     for (int c = 0; c < nch; ++c) {
       const int s = c % kStages, n = c / kStages;
       float* sc = reinterpret_cast<float*>(sm + kOffSc + s * kScFloats * 4);
@@ -402,16 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
         break;
       }
       // gates: G_j by an inclusive scan (tokens 0-31 in warp 0, 32-63 in warp 1)
-      float gj = 0.f, bj = 0.f;
-      if (tid < kC) {
-        const int p = kC * c + tid;
-        if (p < a.P) {
-          const size_t ix = (size_t(r) * a.P + p) * a.H + h;
-          gj = __ldg(a.g + ix);
-          bj = __ldg(a.beta + ix);
-        }
-      }
       float G = gj;
+      const float bcur = bj;
+      load_gates(c + 1, gj, bj);
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float y = __shfl_up_sync(kFull, G, o);
@@ -425,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
       const float GC = Gs[kC - 1];
       if (tid < kC) {
         sc[tid] = expf(G);
-        sc[kC + tid] = bj;
+        sc[kC + tid] = bcur;
         sc[2 * kC + tid] = expf(GC - G);
       }
       if (tid == 0) sc[3 * kC] = expf(GC);
@@ -449,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int m = 16 * q + e;
-              Lm[jr * kLd + m] = m < jr ? bjr * expf(Gj - Gs[m]) * A[e] : 0.f;
+              Lm[jr * kLd + m] = m < jr ? bjr * __expf(Gj - Gs[m]) * A[e] : 0.f;
             }
           }
         }
@@ -462,36 +471,56 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
       // column), then T_ba = -T_bb sum_{a <= c < b} L_bc T_ca by block distance b - a
       if (tid < kC) {
         const int o = 16 * (tid >> 4), m = tid & 15;
+        // right-looking: once x[ii] is final it updates every later row (a chain of 15 steps)
         float x[16];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          float acc = jj == m ? 1.f : 0.f;
+        for (int jj = 0; jj < 16; ++jj) x[jj] = jj == m ? 1.f : 0.f;
 #pragma unroll
-          for (int ii = 0; ii < jj; ++ii) acc -= Lm[(o + jj) * kLd + o + ii] * x[ii];
-          x[jj] = acc;
+        for (int ii = 0; ii < 15; ++ii) {
+#pragma unroll
+          for (int jj = ii + 1; jj < 16; ++jj) x[jj] -= Lm[(o + jj) * kLd + o + ii] * x[ii];
         }
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) Tf[(o + jj) * kLd + o + m] = x[jj];
+        for (int jj = 0; jj < 16; ++jj) Tf[(o + jj) * kLdT + o + m] = x[jj];
       }
       named_bar_sync(kBarPre, 128);
+      // task = (block pair, row y, 4 columns x0..x0+3)
 #pragma unroll 1
       for (int dl = 1; dl < 4; ++dl) {
-        const int nout = (4 - dl) * 256;
-        for (int o = tid; o < nout; o += 128) {
-          const int ab = o >> 8, bb = ab + dl, y = (o >> 4) & 15, x = o & 15;
+        const int ntask = (4 - dl) * 64;
+        for (int o = tid; o < ntask; o += 128) {
+          const int ab = o >> 6, bb = ab + dl, y = (o >> 2) & 15, x0 = (o & 3) * 4;
           const float* lrow = Lm + (16 * bb + y) * kLd;
-          float acc = 0.f;
-#pragma unroll 4
-          for (int ii = 16 * ab; ii < 16 * bb; ++ii) acc += lrow[ii] * Tf[ii * kLd + 16 * ab + x];
-          Qb[o] = acc;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+          for (int cb = ab; cb < bb; ++cb) {
+#pragma unroll
+            for (int z = 0; z < 16; ++z) {
+              const float l = lrow[16 * cb + z];
+              const float4 t = *reinterpret_cast<const float4*>(Tf + (16 * cb + z) * kLdT + 16 * ab + x0);
+              acc.x += l * t.x;
+              acc.y += l * t.y;
+              acc.z += l * t.z;
+              acc.w += l * t.w;
+            }
+          }
+          *reinterpret_cast<float4*>(Qb + (ab * 16 + y) * 16 + x0) = acc;
         }
         named_bar_sync(kBarPre, 128);
-        for (int o = tid; o < nout; o += 128) {
-          const int ab = o >> 8, bb = ab + dl, y = (o >> 4) & 15, x = o & 15;
-          const float* trow = Tf + (16 * bb + y) * kLd + 16 * bb;
-          float acc = 0.f;
-          for (int z = 0; z <= y; ++z) acc -= trow[z] * Qb[(ab << 8) + (z << 4) + x];
-          Tf[(16 * bb + y) * kLd + 16 * ab + x] = acc;
+        for (int o = tid; o < ntask; o += 128) {
+          const int ab = o >> 6, bb = ab + dl, y = (o >> 2) & 15, x0 = (o & 3) * 4;
+          const float* trow = Tf + (16 * bb + y) * kLdT + 16 * bb;   // T_bb row y (0 past the diagonal)
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int z = 0; z < 16; ++z) {
+            const float tz = trow[z];
+            const float4 q = *reinterpret_cast<const float4*>(Qb + (ab * 16 + z) * 16 + x0);
+            acc.x -= tz * q.x;
+            acc.y -= tz * q.y;
+            acc.z -= tz * q.z;
+            acc.w -= tz * q.w;
+          }
+          *reinterpret_cast<float4*>(Tf + (16 * bb + y) * kLdT + 16 * ab + x0) = acc;
         }
         named_bar_sync(kBarPre, 128);
       }
@@ -507,8 +536,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int m0 = 8 * q + 2 * e;
-            const float t0 = m0 <= jr ? Tf[jr * kLd + m0] : 0.f;
-            const float t1 = m0 + 1 <= jr ? Tf[jr * kLd + m0 + 1] : 0.f;
+            const float t0 = m0 <= jr ? Tf[jr * kLdT + m0] : 0.f;
+            const float t1 = m0 + 1 <= jr ? Tf[jr * kLdT + m0 + 1] : 0.f;
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(t0, t1);
             const float2 hf2 = __bfloat1622float2(h2);
             const __nv_bfloat162 l2 = __floats2bfloat162_rn(t0 - hf2.x, t1 - hf2.y);
