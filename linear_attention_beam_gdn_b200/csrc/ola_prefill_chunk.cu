@@ -14,14 +14,14 @@
 // D = diag(e^{G_C - G_j}); rows of S are independent (row i only meets v[i]). Every exponent
 // is a difference G_j - G_m <= 0 or G <= 0, so no factor exceeds 1.
 //
-// One CTA per (request, head), one per SM (tensor memory: 448 of 512 columns):
-//   warps 0-3  per chunk, one chunk ahead of the state chain: gates (prefix sums, a, D), L from
-//              K K^T, T in fp32 by 16 x 16 blocks (diagonal blocks by forward substitution,
+// One CTA per (request, head), one per SM (tensor memory: 384 of 512 columns):
+//   warps 0-3  per chunk, ahead of the state chain: gates (prefix sums, a, D), K K^T on
+//              warp-level MMA from the key tile (exact bf16 products), L, T in fp32 by 16 x 16 blocks (diagonal blocks by forward substitution,
 //              then T_ba = -T_bb sum_{a <= c < b} L_bc T_ca by block distance), T as bf16 hi + lo
 //   warps 4-7  state rows (thread = row = tensor-memory lane): R, W D, and the state entering
 //              the next chunk (its bf16 hi + lo for Z, and a_C S for the accumulation)
 //   warp 8     TMA: key and value tiles of each chunk, three stages
-//   warp 9     tcgen05.mma: K K^T (M = 64), Z = S K^T (S hi + lo in tensor memory),
+//   warp 9     tcgen05.mma: Z = S K^T (S hi + lo in tensor memory),
 //              W = R T^T (three products of hi/lo parts), S += (W D) K (keys as MN-major B)
 // fp32 values enter the tensor cores as hi = bf16(x) plus lo = bf16(x - hi) (about 16
 // significant bits); the lo x lo product is dropped; keys are bf16 already and exact.
@@ -40,14 +40,13 @@ constexpr int kWTma = 8;
 constexpr int kWMma = 9;
 constexpr int kBarPre = 1;         // named barrier of the four precompute warps
 
-// tensor memory columns (lane = state row, or token row of K K^T)
+// tensor memory columns (lane = state row)
 constexpr uint32_t kTS = 0;        // S fp32, 128 columns
 constexpr uint32_t kTSH = 128;     // S as bf16 hi, two per column (64 columns)
 constexpr uint32_t kTSL = 192;     // S as bf16 lo
 constexpr uint32_t kTZ = 256;      // Z, then W: fp32, one column per token (64)
 constexpr uint32_t kTRH = 320;     // R, then W D: bf16 hi (32 columns)
 constexpr uint32_t kTRL = 352;     // ... bf16 lo
-constexpr uint32_t kTG = 384;      // K K^T, M = 64 layout (64 columns)
 
 // shared memory, offsets from a 1024-byte aligned base
 constexpr uint32_t kTile = kC * kD * 2;                        // 16 KB: [2 col blocks][64][128 B]
@@ -64,7 +63,7 @@ constexpr uint32_t kOffTf = kOffL + kC * kLd * 4;              // T fp32 [64][68
 constexpr uint32_t kOffQ = kOffTf + kC * kLdT * 4;             // block products [3][16][16]
 constexpr uint32_t kOffG = kOffQ + 3 * 256 * 4;                // G_j [64] + a warp total
 constexpr uint32_t kOffBar = kOffG + (kC + 4) * 4;
-constexpr int kNumBars = 18;
+constexpr int kNumBars = 16;
 constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + holder, alignment
 static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
 static_assert(kOffTf % 16 == 0 && kOffQ % 16 == 0, "float4 rows of T and of the block products");
@@ -142,15 +141,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
   uint64_t* full = bar;              // [3] key and value tiles landed (TMA bytes)
   uint64_t* empty = bar + 3;         // [3] stage reusable: MMA commit + 4 state-row warps
   uint64_t* pre = bar + 6;           // [3] T tiles and gate scalars written: 4 precompute warps
-  uint64_t* gram_done = bar + 9;     // K K^T in tensor memory
-  uint64_t* gram_free = bar + 10;    // ... read (4 precompute warps)
-  uint64_t* z_full = bar + 11;       // Z in tensor memory
-  uint64_t* r_full = bar + 12;       // R hi/lo written (4 state-row warps)
-  uint64_t* w_full = bar + 13;       // W in tensor memory
-  uint64_t* y_full = bar + 14;       // W D hi/lo written (4 state-row warps)
-  uint64_t* s_full = bar + 15;       // S updated
-  uint64_t* shl_full = bar + 16;     // S hi/lo and a_C S written (4 state-row warps)
-  uint64_t* mma_done = bar + 17;     // every MMA of the CTA completed
+  uint64_t* z_full = bar + 9;        // Z in tensor memory
+  uint64_t* r_full = bar + 10;       // R hi/lo written (4 state-row warps)
+  uint64_t* w_full = bar + 11;       // W in tensor memory
+  uint64_t* y_full = bar + 12;       // W D hi/lo written (4 state-row warps)
+  uint64_t* s_full = bar + 13;       // S updated
+  uint64_t* shl_full = bar + 14;     // S hi/lo and a_C S written (4 state-row warps)
+  uint64_t* mma_done = bar + 15;     // every MMA of the CTA completed
   uint32_t* holder = reinterpret_cast<uint32_t*>(bar + kNumBars);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = blockIdx.x / a.H, h = blockIdx.x % a.H;
@@ -162,8 +159,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
       mbar_init(&empty[s], 5);
       mbar_init(&pre[s], 4);
     }
-    mbar_init(gram_done, 1);
-    mbar_init(gram_free, 4);
     mbar_init(z_full, 1);
     mbar_init(r_full, 4);
     mbar_init(w_full, 1);
@@ -208,24 +203,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
     }
   } else if (warp == kWMma) {
     // ---------------------------------------------------------------- MMA issue
-    const uint32_t id_g = idesc_bf16_f32(64, kC);
     const uint32_t id_z = idesc_bf16_f32(128, kC);
     const uint32_t id_s = idesc_bf16_f32(128, kD) | (1u << 16);     // B (the keys) MN-major
-    bool ok = __all_sync(kFull, mbar_wait_bounded(&full[0], 0));
-    tc_fence_after();
-    if (ok) {
-#pragma unroll 1
-      for (int ks = 0; ks < kD / 16; ++ks) {             // K K^T of chunk 0
-        const uint64_t d = sw128_kmajor_desc(kbase + (ks >> 2) * 8192 + (ks & 3) * 32);
-        umma_bf16_w(tmem + kTG, d, d, id_g, ks != 0);
-      }
-      umma_commit_w(gram_done);
-    }
+    bool ok = true;
     for (int c = 0; c < nch && ok; ++c) {
       const int s = c % kStages, n = c / kStages;
       const uint32_t kb = kbase + s * kTile;
       // Z = S K^T: M = 128 state rows, N = 64 tokens, K = d_k; S as hi + lo from tensor memory
-      ok = __all_sync(kFull, mbar_wait_bounded(shl_full, c & 1));
+      ok = __all_sync(kFull, mbar_wait_bounded(&full[s], n & 1) && mbar_wait_bounded(shl_full, c & 1));
       tc_fence_after();
       if (!ok) break;
 #pragma unroll 1
@@ -235,21 +220,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
         umma_bf16_ts_w(tmem + kTZ, tmem + kTSL + ks * 8, b, id_z, 1u);
       }
       umma_commit_w(z_full);
-      // K K^T of the next chunk, once its keys have landed and this chunk's has been read
-      if (c + 1 < nch) {
-        const int s1 = (c + 1) % kStages;
-        ok = __all_sync(kFull, mbar_wait_bounded(&full[s1], ((c + 1) / kStages) & 1) &&
-                                   mbar_wait_bounded(gram_free, c & 1));
-        tc_fence_after();
-        if (!ok) break;
-#pragma unroll 1
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint64_t d =
-              sw128_kmajor_desc(kbase + s1 * kTile + (ks >> 2) * 8192 + (ks & 3) * 32);
-          umma_bf16_w(tmem + kTG, d, d, id_g, ks != 0);
-        }
-        umma_commit_w(gram_done);
-      }
       // W = R T^T: M = 128, N = 64 tokens, K = 64 tokens; R_hi T_hi + R_hi T_lo + R_lo T_hi
       ok = __all_sync(kFull, mbar_wait_bounded(&pre[s], n & 1) && mbar_wait_bounded(r_full, c & 1));
       tc_fence_after();
@@ -391,7 +361,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
     if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 42, 0);
   } else {
     // ---------------------------------------------------------------- per-chunk precompute
-    const int sp = warp;
     float* Lm = reinterpret_cast<float*>(sm + kOffL);
     float* Tf = reinterpret_cast<float*>(sm + kOffTf);
     float* Qb = reinterpret_cast<float*>(sm + kOffQ);
@@ -438,34 +407,51 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
         sc[2 * kC + tid] = expf(GC - G);
       }
       if (tid == 0) sc[3 * kC] = expf(GC);
-      // L from K K^T: thread (sp, lane < 16) holds row 16 sp + lane (the M = 64 layout puts
-      // rows 16 sp .. 16 sp + 15 in lanes 0-15 of subpartition sp)
-      ok = mbar_wait_bounded(gram_done, c & 1);
+      // K K^T rows 16 w .. 16 w + 15 (warp w) on warp-level MMA from the swizzled key tile, the
+      // 16-column tiles up to the diagonal only, and L from it (entries on or above the
+      // diagonal are never read)
+      ok = mbar_wait_bounded(&full[s], n & 1);
       if (!bar_and(kBarPre, 128, ok)) {
         if (tid == 0) report_error(a.err, OLA_ERR_TIMEOUT, 44, c);
         break;
       }
-      tc_fence_after();
       {
-        const int jr = 16 * sp + (lane & 15);
-        const uint32_t tg = tmem + (uint32_t(32 * sp) << 16) + kTG;
-        const float Gj = Gs[jr], bjr = sc[kC + jr];
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          float A[16];
-          tmem_ld16(tg + 16 * q, A);
-          if (lane < 16) {
+        const uint32_t kt = smem_u32(sm + kOffK + s * kTile);
+        // byte of the 8 keys columns x .. x + 7 of token t in the tile
+        auto kaddr = [&](int t, int x) {
+          return kt + uint32_t(x >> 6) * 8192u + uint32_t(t) * 128u +
+                 uint32_t((((x & 63) >> 3) ^ (t & 7)) << 4);
+        };
+        const int jb = warp;
+        uint32_t af[8][4];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int m = 16 * q + e;
-              Lm[jr * kLd + m] = m < jr ? bjr * __expf(Gj - Gs[m]) * A[e] : 0.f;
-            }
+        for (int ks = 0; ks < 8; ++ks)
+          ldsm_x4(kaddr(16 * jb + (lane & 15), 16 * ks + (lane >> 4) * 8), af[ks][0], af[ks][1],
+                  af[ks][2], af[ks][3]);
+        const int j0 = 16 * jb + (lane >> 2), j1 = j0 + 8, cq = 2 * (lane & 3);
+        const float G0 = Gs[j0], G1 = Gs[j1], b0 = sc[kC + j0], b1 = sc[kC + j1];
+        const int bt = ((lane >> 3) >> 1) * 8 + (lane & 7), bx = ((lane >> 3) & 1) * 8;
+#pragma unroll 1
+        for (int mp = 0; mp <= jb; ++mp) {
+          float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            uint32_t b00, b01, b10, b11;
+            ldsm_x4(kaddr(16 * mp + bt, 16 * ks + bx), b00, b01, b10, b11);
+            mma_16816_bf16(d0, af[ks][0], af[ks][1], af[ks][2], af[ks][3], b00, b01);
+            mma_16816_bf16(d1, af[ks][0], af[ks][1], af[ks][2], af[ks][3], b10, b11);
+          }
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int m = 16 * mp + cq + e, m8 = m + 8;
+            const float Gm = Gs[m], Gm8 = Gs[m8];
+            Lm[j0 * kLd + m] = m < j0 ? b0 * __expf(G0 - Gm) * d0[e] : 0.f;
+            Lm[j1 * kLd + m] = m < j1 ? b1 * __expf(G1 - Gm) * d0[2 + e] : 0.f;
+            Lm[j0 * kLd + m8] = m8 < j0 ? b0 * __expf(G0 - Gm8) * d1[e] : 0.f;
+            Lm[j1 * kLd + m8] = m8 < j1 ? b1 * __expf(G1 - Gm8) * d1[2 + e] : 0.f;
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(gram_free);
       named_bar_sync(kBarPre, 128);
       // T = (I + L)^-1: the four 16 x 16 diagonal blocks by forward substitution (thread =
       // column), then T_ba = -T_bb sum_{a <= c < b} L_bc T_ca by block distance b - a
