@@ -15,7 +15,7 @@
 // is a difference G_j - G_m <= 0 or G <= 0, so no factor exceeds 1.
 //
 // One CTA per (request, head), one per SM (tensor memory: 384 of 512 columns):
-//   warps 0-3  per chunk, ahead of the state chain: gates (prefix sums, a, D), K K^T on
+//   warps 0-3 and 10-13: two groups taking alternate chunks, ahead of the state chain: gates (prefix sums, a, D), K K^T on
 //              warp-level MMA from the key tile (exact bf16 products), L, T in fp32 by 16 x 16 blocks (diagonal blocks by forward substitution,
 //              then T_ba = -T_bb sum_{a <= c < b} L_bc T_ca by block distance), T as bf16 hi + lo
 //   warps 4-7  state rows (thread = row = tensor-memory lane): R, W D, and the state entering
@@ -34,11 +34,12 @@ namespace {
 constexpr int kC = 64;             // tokens per chunk
 constexpr int kD = 128;            // d_k = d_v
 constexpr int kStages = 3;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr int kWRow = 4;           // first state-row warp
 constexpr int kWTma = 8;
 constexpr int kWMma = 9;
-constexpr int kBarPre = 1;         // named barrier of the four precompute warps
+constexpr int kWPre1 = 10;         // first warp of the second precompute group
+constexpr int kBarPre = 1;         // named barriers 1 and 2: the two precompute groups
 
 // tensor memory columns (lane = state row)
 constexpr uint32_t kTS = 0;        // S fp32, 128 columns
@@ -58,15 +59,18 @@ constexpr uint32_t kOffK = 0;                                  // keys, 128-byte
 constexpr uint32_t kOffV = kOffK + kStages * kTile;            // values, no swizzle
 constexpr uint32_t kOffT = kOffV + kStages * kTile;            // T hi, T lo per stage
 constexpr uint32_t kOffSc = kOffT + kStages * 2 * kTTile;      // gate scalars per stage
-constexpr uint32_t kOffL = kOffSc + kStages * kScFloats * 4;   // L fp32 [64][65]
-constexpr uint32_t kOffTf = kOffL + kC * kLd * 4;              // T fp32 [64][68]
-constexpr uint32_t kOffQ = kOffTf + kC * kLdT * 4;             // block products [3][16][16]
-constexpr uint32_t kOffG = kOffQ + 3 * 256 * 4;                // G_j [64] + a warp total
-constexpr uint32_t kOffBar = kOffG + (kC + 4) * 4;
+constexpr uint32_t kOffGrp = kOffSc + kStages * kScFloats * 4; // per precompute group:
+constexpr uint32_t kGL = 0;                                    //   L fp32 [64][65]
+constexpr uint32_t kGTf = kGL + kC * kLd * 4;                  //   T fp32 [64][68]
+constexpr uint32_t kGQ = kGTf + kC * kLdT * 4;                 //   block products [3][16][16]
+constexpr uint32_t kGG = kGQ + 3 * 256 * 4;                    //   G_j [64] + a warp total
+constexpr uint32_t kGrpBytes = kGG + (kC + 4) * 4;
+constexpr uint32_t kOffBar = kOffGrp + 2 * kGrpBytes;
 constexpr int kNumBars = 16;
 constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + holder, alignment
 static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
-static_assert(kOffTf % 16 == 0 && kOffQ % 16 == 0, "float4 rows of T and of the block products");
+static_assert((kOffGrp + kGTf) % 16 == 0 && (kOffGrp + kGQ) % 16 == 0 && kGrpBytes % 16 == 0,
+              "float4 rows of T and of the block products");
 static_assert(kOffT % 1024 == 0 && kOffV % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
@@ -252,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
     umma_commit_w(mma_done);
     mbar_wait_bounded(mma_done, 0);
     __syncwarp();
-  } else if (warp >= kWRow) {
+  } else if (warp >= kWRow && warp < kWRow + 4) {
     // ---------------------------------------------------------------- state rows
     const int sp = warp & 3, i = 32 * sp + lane;
     const uint32_t tl = tmem + (uint32_t(32 * sp) << 16);
@@ -361,58 +365,62 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
     if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 42, 0);
   } else {
     // ---------------------------------------------------------------- per-chunk precompute
-    float* Lm = reinterpret_cast<float*>(sm + kOffL);
-    float* Tf = reinterpret_cast<float*>(sm + kOffTf);
-    float* Qb = reinterpret_cast<float*>(sm + kOffQ);
-    float* Gs = reinterpret_cast<float*>(sm + kOffG);
+    // group grp takes chunks grp, grp + 2, ...; ptid = thread, pw = warp within the group
+    const int grp = warp >= kWPre1 ? 1 : 0;
+    const int ptid = tid - 32 * (grp ? kWPre1 : 0), pw = ptid >> 5, pbar = kBarPre + grp;
+    unsigned char* gb = sm + kOffGrp + grp * kGrpBytes;
+    float* Lm = reinterpret_cast<float*>(gb + kGL);
+    float* Tf = reinterpret_cast<float*>(gb + kGTf);
+    float* Qb = reinterpret_cast<float*>(gb + kGQ);
+    float* Gs = reinterpret_cast<float*>(gb + kGG);
     // gates of chunk c (tokens past P: g = 0, beta = 0, an identity step), loaded a chunk ahead
     auto load_gates = [&](int c, float& gv, float& bv) {
       gv = 0.f;
       bv = 0.f;
-      const int p = kC * c + tid;
-      if (tid < kC && c < nch && p < a.P) {
+      const int p = kC * c + ptid;
+      if (ptid < kC && c < nch && p < a.P) {
         const size_t ix = (size_t(r) * a.P + p) * a.H + h;
         gv = __ldg(a.g + ix);
         bv = __ldg(a.beta + ix);
       }
     };
     float gj, bj;
-    load_gates(0, gj, bj);
-    for (int c = 0; c < nch; ++c) {
+    load_gates(grp, gj, bj);
+    for (int c = grp; c < nch; c += 2) {
       const int s = c % kStages, n = c / kStages;
       float* sc = reinterpret_cast<float*>(sm + kOffSc + s * kScFloats * 4);
       bool ok = n == 0 || mbar_wait_bounded(&empty[s], (n - 1) & 1);
-      if (!bar_and(kBarPre, 128, ok)) {
-        if (tid == 0) report_error(a.err, OLA_ERR_TIMEOUT, 43, c);
+      if (!bar_and(pbar, 128, ok)) {
+        if (ptid == 0) report_error(a.err, OLA_ERR_TIMEOUT, 43, c);
         break;
       }
-      // gates: G_j by an inclusive scan (tokens 0-31 in warp 0, 32-63 in warp 1)
+      // gates: G_j by an inclusive scan (tokens 0-31 in the group's warp 0, 32-63 in its warp 1)
       float G = gj;
       const float bcur = bj;
-      load_gates(c + 1, gj, bj);
+      load_gates(c + 2, gj, bj);
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float y = __shfl_up_sync(kFull, G, o);
         if (lane >= o) G += y;
       }
-      if (tid == 31) Gs[kC] = G;
-      named_bar_sync(kBarPre, 128);
-      if (tid >= 32 && tid < kC) G += Gs[kC];
-      if (tid < kC) Gs[tid] = G;
-      named_bar_sync(kBarPre, 128);
+      if (ptid == 31) Gs[kC] = G;
+      named_bar_sync(pbar, 128);
+      if (ptid >= 32 && ptid < kC) G += Gs[kC];
+      if (ptid < kC) Gs[ptid] = G;
+      named_bar_sync(pbar, 128);
       const float GC = Gs[kC - 1];
-      if (tid < kC) {
-        sc[tid] = expf(G);
-        sc[kC + tid] = bcur;
-        sc[2 * kC + tid] = expf(GC - G);
+      if (ptid < kC) {
+        sc[ptid] = expf(G);
+        sc[kC + ptid] = bcur;
+        sc[2 * kC + ptid] = expf(GC - G);
       }
-      if (tid == 0) sc[3 * kC] = expf(GC);
-      // K K^T rows 16 w .. 16 w + 15 (warp w) on warp-level MMA from the swizzled key tile, the
+      if (ptid == 0) sc[3 * kC] = expf(GC);
+      // K K^T rows 16 w .. 16 w + 15 (group warp w) on warp-level MMA from the swizzled key tile, the
       // 16-column tiles up to the diagonal only, and L from it (entries on or above the
       // diagonal are never read)
       ok = mbar_wait_bounded(&full[s], n & 1);
-      if (!bar_and(kBarPre, 128, ok)) {
-        if (tid == 0) report_error(a.err, OLA_ERR_TIMEOUT, 44, c);
+      if (!bar_and(pbar, 128, ok)) {
+        if (ptid == 0) report_error(a.err, OLA_ERR_TIMEOUT, 44, c);
         break;
       }
       {
@@ -422,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
           return kt + uint32_t(x >> 6) * 8192u + uint32_t(t) * 128u +
                  uint32_t((((x & 63) >> 3) ^ (t & 7)) << 4);
         };
-        const int jb = warp;
+        const int jb = pw;
         uint32_t af[8][4];
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
@@ -452,11 +460,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
           }
         }
       }
-      named_bar_sync(kBarPre, 128);
+      named_bar_sync(pbar, 128);
       // T = (I + L)^-1: the four 16 x 16 diagonal blocks by forward substitution (thread =
       // column), then T_ba = -T_bb sum_{a <= c < b} L_bc T_ca by block distance b - a
-      if (tid < kC) {
-        const int o = 16 * (tid >> 4), m = tid & 15;
+      if (ptid < kC) {
+        const int o = 16 * (ptid >> 4), m = ptid & 15;
         // right-looking: once x[ii] is final it updates every later row (a chain of 15 steps)
         float x[16];
 #pragma unroll
@@ -469,12 +477,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) Tf[(o + jj) * kLdT + o + m] = x[jj];
       }
-      named_bar_sync(kBarPre, 128);
+      named_bar_sync(pbar, 128);
       // task = (block pair, row y, 4 columns x0..x0+3)
 #pragma unroll 1
       for (int dl = 1; dl < 4; ++dl) {
         const int ntask = (4 - dl) * 64;
-        for (int o = tid; o < ntask; o += 128) {
+        for (int o = ptid; o < ntask; o += 128) {
           const int ab = o >> 6, bb = ab + dl, y = (o >> 2) & 15, x0 = (o & 3) * 4;
           const float* lrow = Lm + (16 * bb + y) * kLd;
           float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -492,8 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
           }
           *reinterpret_cast<float4*>(Qb + (ab * 16 + y) * 16 + x0) = acc;
         }
-        named_bar_sync(kBarPre, 128);
-        for (int o = tid; o < ntask; o += 128) {
+        named_bar_sync(pbar, 128);
+        for (int o = ptid; o < ntask; o += 128) {
           const int ab = o >> 6, bb = ab + dl, y = (o >> 2) & 15, x0 = (o & 3) * 4;
           const float* trow = Tf + (16 * bb + y) * kLdT + 16 * bb;   // T_bb row y (0 past the diagonal)
           float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -508,11 +516,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
           }
           *reinterpret_cast<float4*>(Tf + (16 * bb + y) * kLdT + 16 * ab + x0) = acc;
         }
-        named_bar_sync(kBarPre, 128);
+        named_bar_sync(pbar, 128);
       }
       // T as bf16 hi and lo, K-major tiles with the 128-byte swizzle: thread = half a row
       {
-        const int jr = tid >> 1, hf = tid & 1;
+        const int jr = ptid >> 1, hf = ptid & 1;
         unsigned char* thi = sm + kOffT + s * 2 * kTTile;
         unsigned char* tlo = thi + kTTile;
 #pragma unroll
