@@ -299,6 +299,7 @@ def run_ours(args):
     # ---- inputs resident in HBM; shared state by the library's prefill kernel
     prompt = wl.make_prompt(w, dev)
     S = ola.prefill(prompt["k"], prompt["v"], prompt["g"], prompt["beta"])
+    pf_ms = time_prefill(prompt)
     steps = [wl.make_step_inputs(w, t, dev) for t in range(w.T)]
     parents = wl.make_parents(w)
     par_dev = [torch.from_numpy(parents[t]).to(dev) for t in range(w.T)]
@@ -382,6 +383,13 @@ def run_ours(args):
                          "parallelism": f"replicas x{world} (requests sharded, no collective)"},
               "roofline": roofline, "clocks": clocks,
               "gpu_launches": 2 * w.T * K}
+    pf_bytes = prefill_bytes(w)
+    result["prefill"] = {
+        "what": "shared state from the prompt (once per request batch, outside the timed "
+                "decode steps); chunked tensor-core form for 128x128 bf16, else token by token",
+        "ms": pf_ms, "algorithmic_bytes": pf_bytes,
+        "achieved_gbs": pf_bytes / (pf_ms / 1e3) / 1e9,
+        "hbm_frac": pf_bytes / (pf_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
 
     # ---- in-library comparisons on the same inputs (not part of the metric)
     comps = {}
@@ -469,6 +477,31 @@ SWEEP_REQUESTS = (1, 2, 8, 32, 64)
 SWEEP_BEAMS = (64, 256, 512)
 SWEEP_STEPS = (2, 4, 8)
 SWEEP_FULLSTATE_LIMIT = 96 << 30      # bytes of FullState ping-pong state the sweep allocates
+
+
+def prefill_bytes(w: wl.Workload) -> int:
+    """Bytes the prefill must move: the prompt's k, v (input dtype), g and beta (fp32) read
+    once, the fp32 state of every (request, head) written once."""
+    e = 2 if w.dtype == "bf16" else 4
+    return w.R * w.P * w.H * ((w.d_k + w.d_v) * e + 8) + w.R * w.H * w.d_v * w.d_k * 4
+
+
+def time_prefill(prompt, reps: int = 5) -> float:
+    """Median device time (ms, CUDA events) of ola.prefill on the resident prompt."""
+    import torch
+    import linear_attention_beam_gdn_b200 as ola
+    for _ in range(2):                                   # warm-up
+        ola.prefill(prompt["k"], prompt["v"], prompt["g"], prompt["beta"])
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        ola.prefill(prompt["k"], prompt["v"], prompt["g"], prompt["beta"])
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return float(np.median(ts))
 
 
 def fullstate_bytes_per_step(w: wl.Workload, parents: np.ndarray) -> list:

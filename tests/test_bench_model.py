@@ -46,3 +46,13 @@ def test_replay_bytes_grow_with_distinct_ancestors():
     assert a[0] == b[0]
     # step 3: one ancestor per slot with a single parent line, four per slot when spread
     assert b[2] - a[2] == w.H * (8 - 2) * rec
+
+
+def test_prefill_bytes_are_the_prompt_tensors_plus_the_state():
+    """The prefill's byte model counts each prompt tensor once (as generated) and the fp32
+    state once."""
+    for name in ("tiny", "single_request"):
+        w = wl.WORKLOADS[name].scaled(P=40)
+        prompt = wl.make_prompt(w, "cpu")
+        nbytes = sum(t.numel() * t.element_size() for t in prompt.values())
+        assert bench.prefill_bytes(w) == nbytes + w.R * w.H * w.d_v * w.d_k * 4
