@@ -288,9 +288,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
         float x[32];
         tmem_ld32(tl + kTZ + 32 * q, x);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int j = 32 * q + e;
-          x[e] = sc[kC + j] * (__bfloat162float(vt[j * 64]) - sc[j] * x[e]);
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const int j = 32 * q + 4 * e4;
+          const float4 av = *reinterpret_cast<const float4*>(sc + j);
+          const float4 bv = *reinterpret_cast<const float4*>(sc + kC + j);
+          x[4 * e4] = bv.x * (__bfloat162float(vt[j * 64]) - av.x * x[4 * e4]);
+          x[4 * e4 + 1] = bv.y * (__bfloat162float(vt[(j + 1) * 64]) - av.y * x[4 * e4 + 1]);
+          x[4 * e4 + 2] = bv.z * (__bfloat162float(vt[(j + 2) * 64]) - av.z * x[4 * e4 + 2]);
+          x[4 * e4 + 3] = bv.w * (__bfloat162float(vt[(j + 3) * 64]) - av.w * x[4 * e4 + 3]);
         }
         uint4 hi[4], lo[4];
         split32(x, hi, lo);
@@ -310,7 +315,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
         float x[32];
         tmem_ld32(tl + kTZ + 32 * q, x);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] *= sc[2 * kC + 32 * q + e];
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 dv = *reinterpret_cast<const float4*>(sc + 2 * kC + 32 * q + 4 * e4);
+          x[4 * e4] *= dv.x;
+          x[4 * e4 + 1] *= dv.y;
+          x[4 * e4 + 2] *= dv.z;
+          x[4 * e4 + 3] *= dv.w;
+        }
         uint4 hi[4], lo[4];
         split32(x, hi, lo);
         tmem_st16(tl + kTRH + 16 * q, hi);
@@ -331,8 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
       if (!__all_sync(kFull, ok)) break;
       tc_fence_after();
       if (!last) {
-        const float aC =
-            reinterpret_cast<const float*>(sm + kOffSc + s1 * kScFloats * 4)[3 * kC];
+        // hi + lo for the next Z first (the chain waits on them), then a_C S for the next
+        // accumulation, which overlaps the next Z
 #pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           float x[32];
@@ -341,14 +352,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
           split32(x, hi, lo);
           tmem_st16(tl + kTSH + 16 * q, hi);
           tmem_st16(tl + kTSL + 16 * q, lo);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] *= aC;
-          tmem_st32(tl + kTS + 32 * q, x);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(shl_full);
+        const float aC =
+            reinterpret_cast<const float*>(sm + kOffSc + s1 * kScFloats * 4)[3 * kC];
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          float x[32];
+          tmem_ld32(tl + kTS + 32 * q, x);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] *= aC;
+          tmem_st32(tl + kTS + 32 * q, x);
+        }
+        tmem_st_wait();
       } else {
         float* dst = a.S + ((size_t(r) * a.H + h) * kD + i) * size_t(kD);
 #pragma unroll 1
@@ -439,16 +458,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
         const int j0 = 16 * jb + (lane >> 2), j1 = j0 + 8, cq = 2 * (lane & 3);
         const float G0 = Gs[j0], G1 = Gs[j1], b0 = sc[kC + j0], b1 = sc[kC + j1];
         const int bt = ((lane >> 3) >> 1) * 8 + (lane & 7), bx = ((lane >> 3) & 1) * 8;
-#pragma unroll 1
-        for (int mp = 0; mp <= jb; ++mp) {
-          float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+        // the column tiles of the row block accumulate side by side: 2 (jb + 1) independent
+        // MMA chains of 8 steps instead of one long chain
+        float d[4][2][4];
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            uint32_t b00, b01, b10, b11;
-            ldsm_x4(kaddr(16 * mp + bt, 16 * ks + bx), b00, b01, b10, b11);
-            mma_16816_bf16(d0, af[ks][0], af[ks][1], af[ks][2], af[ks][3], b00, b01);
-            mma_16816_bf16(d1, af[ks][0], af[ks][1], af[ks][2], af[ks][3], b10, b11);
+        for (int mp = 0; mp < 4; ++mp)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d[mp][0][e] = d[mp][1][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+          for (int mp = 0; mp < 4; ++mp) {
+            if (mp <= jb) {                              // warp-uniform
+              uint32_t b00, b01, b10, b11;
+              ldsm_x4(kaddr(16 * mp + bt, 16 * ks + bx), b00, b01, b10, b11);
+              mma_16816_bf16(d[mp][0], af[ks][0], af[ks][1], af[ks][2], af[ks][3], b00, b01);
+              mma_16816_bf16(d[mp][1], af[ks][0], af[ks][1], af[ks][2], af[ks][3], b10, b11);
+            }
           }
+        }
+#pragma unroll
+        for (int mp = 0; mp < 4; ++mp) {
+          if (mp > jb) break;
+          const float* d0 = d[mp][0];
+          const float* d1 = d[mp][1];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int m = 16 * mp + cq + e, m8 = m + 8;
