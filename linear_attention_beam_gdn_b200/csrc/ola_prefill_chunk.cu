@@ -15,9 +15,11 @@
 // is a difference G_j - G_m <= 0 or G <= 0, so no factor exceeds 1.
 //
 // One CTA per (request, head), one per SM (tensor memory: 384 of 512 columns):
-//   warps 0-3 and 10-13: two groups taking alternate chunks, ahead of the state chain: gates (prefix sums, a, D), K K^T on
-//              warp-level MMA from the key tile (exact bf16 products), L, T in fp32 by 16 x 16 blocks (diagonal blocks by forward substitution,
-//              then T_ba = -T_bb sum_{a <= c < b} L_bc T_ca by block distance), T as bf16 hi + lo
+//   warps 0-3, 10-13  two precompute groups taking alternate chunks, ahead of the state
+//              chain: gates (prefix sums, a, D), K K^T on warp-level MMA from the key tile
+//              (exact bf16 products), L, T in fp32 by 16 x 16 blocks (diagonal blocks by
+//              forward substitution, then T_ba = -T_bb sum_{a <= c < b} L_bc T_ca by block
+//              distance), T as bf16 hi + lo tiles
 //   warps 4-7  state rows (thread = row = tensor-memory lane): R, W D, and the state entering
 //              the next chunk (its bf16 hi + lo for Z, and a_C S for the accumulation)
 //   warp 8     TMA: key and value tiles of each chunk, three stages
