@@ -140,7 +140,8 @@ __device__ __forceinline__ void tmem_st32(uint32_t t, const float (&x)[32]) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid_constant__ ChunkArgs a) {
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_chunk_kernel(const __grid_constant__ ChunkArgs a) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = align_smem_1024(smem_raw);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kOffBar);
@@ -216,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
       const int s = c % kStages, n = c / kStages;
       const uint32_t kb = kbase + s * kTile;
       // Z = S K^T: M = 128 state rows, N = 64 tokens, K = d_k; S as hi + lo from tensor memory
-      ok = __all_sync(kFull, mbar_wait_bounded(&full[s], n & 1) && mbar_wait_bounded(shl_full, c & 1));
+      ok = __all_sync(kFull, mbar_wait_bounded(&full[s], n & 1) &&
+                                 mbar_wait_bounded(shl_full, c & 1));
       tc_fence_after();
       if (!ok) break;
 #pragma unroll 1
@@ -436,9 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
         sc[2 * kC + ptid] = expf(GC - G);
       }
       if (ptid == 0) sc[3 * kC] = expf(GC);
-      // K K^T rows 16 w .. 16 w + 15 (group warp w) on warp-level MMA from the swizzled key tile, the
-      // 16-column tiles up to the diagonal only, and L from it (entries on or above the
-      // diagonal are never read)
+      // K K^T rows 16 w .. 16 w + 15 (group warp w) on warp-level MMA from the swizzled key
+      // tile, the 16-column tiles up to the diagonal only, and L from it (entries on or above
+      // the diagonal are never read)
       ok = mbar_wait_bounded(&full[s], n & 1);
       if (!bar_and(pbar, 128, ok)) {
         if (ptid == 0) report_error(a.err, OLA_ERR_TIMEOUT, 44, c);
@@ -526,7 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
 #pragma unroll
             for (int z = 0; z < 16; ++z) {
               const float l = lrow[16 * cb + z];
-              const float4 t = *reinterpret_cast<const float4*>(Tf + (16 * cb + z) * kLdT + 16 * ab + x0);
+              const float4 t =
+                  *reinterpret_cast<const float4*>(Tf + (16 * cb + z) * kLdT + 16 * ab + x0);
               acc.x += l * t.x;
               acc.y += l * t.y;
               acc.z += l * t.z;
@@ -538,7 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_chunk_kernel(const __grid
         named_bar_sync(pbar, 128);
         for (int o = ptid; o < ntask; o += 128) {
           const int ab = o >> 6, bb = ab + dl, y = (o >> 2) & 15, x0 = (o & 3) * 4;
-          const float* trow = Tf + (16 * bb + y) * kLdT + 16 * bb;   // T_bb row y (0 past the diagonal)
+          // T_bb row y (zeros past the diagonal)
+          const float* trow = Tf + (16 * bb + y) * kLdT + 16 * bb;
           float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
           for (int z = 0; z < 16; ++z) {
