@@ -56,3 +56,17 @@ def test_prefill_bytes_are_the_prompt_tensors_plus_the_state():
         prompt = wl.make_prompt(w, "cpu")
         nbytes = sum(t.numel() * t.element_size() for t in prompt.values())
         assert bench.prefill_bytes(w) == nbytes + w.R * w.H * w.d_v * w.d_k * 4
+
+
+def test_state_and_record_bytes_are_the_full_bytes_minus_the_io():
+    """The narrower byte count differs from the full one by exactly the per-beam inputs and
+    outputs and the parent and chain rows."""
+    w = wl.WORKLOADS["single_request"].scaled(R=3, B=16, T=4)
+    parents = wl.make_parents(w)
+    full = bench.algorithmic_bytes_per_step(w, parents)
+    lit = bench.state_and_record_bytes_per_step(w, parents)
+    e = w.elem_bytes
+    for t in range(w.T):
+        io = w.R * w.H * w.B * ((2 * w.d_k + w.d_v) * e + 8 + 4 * w.d_v)
+        rows = w.R * 4 * w.B * (t + 2)
+        assert full[t] - lit[t] == io + rows
