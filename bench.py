@@ -309,13 +309,11 @@ def run_ours(args):
     # ---- inputs resident in HBM; shared state by the library's prefill kernel
     prompt = wl.make_prompt(w, dev)
     S = ola.prefill(prompt["k"], prompt["v"], prompt["g"], prompt["beta"])
-    pf_ms = time_prefill(prompt)
     steps = [wl.make_step_inputs(w, t, dev) for t in range(w.T)]
     parents = wl.make_parents(w)
     par_dev = [torch.from_numpy(parents[t]).to(dev) for t in range(w.T)]
     units = sample_units(w, max(2, 2 * cores)) if do_cpu else []
     host = host_units(w, prompt, steps, parents, units) if do_cpu else None
-    del prompt
     torch.cuda.synchronize()
 
     outs = [torch.empty((w.R, w.B, w.H, w.d_v), device=dev) for _ in range(w.T)]
@@ -396,13 +394,6 @@ def run_ours(args):
                          "parallelism": f"replicas x{world} (requests sharded, no collective)"},
               "roofline": roofline, "clocks": clocks,
               "gpu_launches": 2 * w.T * K}
-    pf_bytes = prefill_bytes(w)
-    result["prefill"] = {
-        "what": "shared state from the prompt (once per request batch, outside the timed "
-                "decode steps); chunked tensor-core form for 128x128 bf16, else token by token",
-        "ms": pf_ms, "algorithmic_bytes": pf_bytes,
-        "achieved_gbs": pf_bytes / (pf_ms / 1e3) / 1e9,
-        "hbm_frac": pf_bytes / (pf_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
 
     # ---- in-library comparisons on the same inputs (not part of the metric)
     comps = {}
@@ -470,11 +461,23 @@ def run_ours(args):
         pu, su, pa = host
         dt, n = oracle_sample(w, pu, su, pa, pool, cores)
         pool.close()
+        pool.join()
         result["cpu_baseline"] = {
             "value": n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{len(pu)} of {w.R * w.H} (request, head) units of this workload, all "
                       f"{w.B} beams x {w.T} steps, fp64 full-state recurrence; the units' "
                       f"fp64 prefill untimed", "seconds": dt}
+
+    # ---- the prompt prefill on its own (after the oracle's host processes have finished:
+    # the chunked form waits for its kernel inside the call, so host load would show)
+    pf_ms = time_prefill(prompt)
+    pf_bytes = prefill_bytes(w)
+    result["prefill"] = {
+        "what": "shared state from the prompt (once per request batch, outside the timed "
+                "decode steps); chunked tensor-core form for 128x128 bf16, else token by token",
+        "ms": pf_ms, "algorithmic_bytes": pf_bytes,
+        "achieved_gbs": pf_bytes / (pf_ms / 1e3) / 1e9,
+        "hbm_frac": pf_bytes / (pf_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
 
     if rank == 0:
         print(json.dumps(result), flush=True)

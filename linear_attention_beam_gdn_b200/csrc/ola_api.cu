@@ -6,6 +6,7 @@
 #include <new>
 
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "ola_device.cuh"
@@ -90,6 +91,13 @@ struct ola_ctx {
 };
 
 namespace {
+
+// Error word of the chunked prefill, one per device, allocated on first use and kept: a
+// per-call stream-ordered allocation would map and unmap pool memory around every call.
+constexpr int kMaxDevices = 64;
+std::mutex g_prefill_mu;
+int* g_prefill_err_dev[kMaxDevices] = {};
+int* g_prefill_err_host[kMaxDevices] = {};
 
 bool pow2_width(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
 bool tc_width(int d) { return d == 64 || d == 128 || d == 256; }
@@ -568,16 +576,27 @@ ola_status ola_prefill(int32_t R, int32_t H, int32_t d_k, int32_t d_v, int32_t P
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (P > 0 && prefill_chunk_supported(d_k, d_v, in_dtype, k, v)) {
     // chunked tensor-core form; waits for it so that a device-side timeout is returned
-    int* derr = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void**>(&derr), 4 * sizeof(int), st) != cudaSuccess)
-      return OLA_ERR_OOM;
-    int herr[4] = {0, 0, 0, 0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return OLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_prefill_mu);
+    if (!g_prefill_err_dev[dev] || !g_prefill_err_host[dev]) {
+      int* d = nullptr;
+      int* hh = nullptr;
+      if (cudaMalloc(reinterpret_cast<void**>(&d), 4 * sizeof(int)) != cudaSuccess)
+        return OLA_ERR_OOM;
+      if (cudaMallocHost(reinterpret_cast<void**>(&hh), 4 * sizeof(int)) != cudaSuccess) {
+        cudaFree(d);
+        return OLA_ERR_OOM;
+      }
+      g_prefill_err_dev[dev] = d;
+      g_prefill_err_host[dev] = hh;
+    }
+    int* derr = g_prefill_err_dev[dev];
+    int* herr = g_prefill_err_host[dev];
     cudaError_t e = cudaMemsetAsync(derr, 0, 4 * sizeof(int), st);
     if (e == cudaSuccess) e = launch_prefill_chunk(R, H, P, k, v, g, beta, S_out, derr, st);
     if (e == cudaSuccess)
-      e = cudaMemcpyAsync(herr, derr, sizeof(herr), cudaMemcpyDeviceToHost, st);
-    const cudaError_t ef = cudaFreeAsync(derr, st);
-    if (e == cudaSuccess) e = ef;
+      e = cudaMemcpyAsync(herr, derr, 4 * sizeof(int), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return from_cuda(e);
     return herr[0] != 0 ? static_cast<ola_status>(herr[0]) : OLA_OK;
