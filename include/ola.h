@@ -194,8 +194,9 @@ ola_status ola_destroy(ola_handle h);
  * d_k, d_v in {16, 32, 64, 128, 256}; P >= 0 (P = 0 writes zeros).
  * d_k = d_v = 128 with a bf16 prompt (k, v 16-byte aligned) runs the chunked tensor-core form
  * (64 tokens per chunk, one CTA per (request, head)) and returns once it has finished, so that
- * a device-side wait that ran out is returned as OLA_ERR_TIMEOUT; every other shape runs token
- * by token on CUDA cores and returns after the launch (stream-ordered).
+ * a device-side wait that ran out is returned as OLA_ERR_TIMEOUT (such calls from several host
+ * threads run one at a time: they share one device error word per device); every other shape
+ * runs token by token on CUDA cores and returns after the launch (stream-ordered).
  * Errors: INVALID_ARG, UNSUPPORTED, OOM, TIMEOUT, CUDA. */
 ola_status ola_prefill(int32_t R, int32_t H, int32_t d_k, int32_t d_v, int32_t P,
                        int32_t in_dtype, const void* k, const void* v, const float* g,

@@ -170,8 +170,8 @@ replay_pos_kernel(const __grid_constant__ CUtensorMap tm_shi,
   const uint32_t tmem = *holder;
 
   // -------------------------------------------------------------------- phase 1
-  // Round 1: the beams of this warp's positions and their parents' chains (both indexed by
-  // position). Round 2: q_t, k_t rows, g, beta, the chain's alphas.
+  // Phase 1: the beams of this warp's positions and their parents' chains (both indexed by
+  // position). Phase 2: q_t, k_t rows, g, beta, the chain's alphas.
   int recs[PPW];
 #pragma unroll
   for (int jj = 0; jj < PPW; ++jj) {
