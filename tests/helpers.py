@@ -85,5 +85,13 @@ def oracle_outputs(S32: torch.Tensor, steps, parents, units=None) -> np.ndarray:
 
 
 def max_abs(a: np.ndarray, b: np.ndarray) -> float:
-    d = np.abs(a - b)
-    return float(np.nanmax(d)) if d.size else 0.0
+    """Largest |a - b| over the positions where the reference b is defined (b holds NaN for
+    units the oracle did not compute); a non-finite a at such a position is an infinite error,
+    so unwritten (NaN-filled) or overflowed outputs never pass."""
+    a, b = np.asarray(a), np.asarray(b)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    mask = np.isfinite(b)
+    if not np.all(np.isfinite(a[mask])):
+        return float("inf")
+    d = np.abs(a[mask] - b[mask])
+    return float(d.max()) if d.size else 0.0

@@ -213,6 +213,7 @@ def test_replay_agrees_with_fullstate_on_gpu():
     S32, steps, dev_steps, parents = small_problem(w)
     o_fs, _, _ = run_library(S32.cuda(), dev_steps, parents, "fullstate", w.torch_dtype)
     o_rp, _, _ = run_library(S32.cuda(), dev_steps, parents, "replay_fp32", w.torch_dtype)
+    assert np.isfinite(o_rp).all()
     assert max_abs(o_fs, o_rp) <= 1e-4
 
 
