@@ -114,10 +114,18 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "10"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return self
+        # nvidia-smi needs a moment before its first sample: start the timed region only once
+        # it is sampling, so that a short region (tens of ms) still gets samples of its own
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.01)
         return self
 
     def __exit__(self, *exc):
@@ -258,6 +266,12 @@ def rank_workload(base: wl.Workload, rank: int) -> wl.Workload:
     return base.scaled(seed=base.seed + 7919 * rank)
 
 
+def job_value(world: int, units_per_rank_step: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: the units every rank processed in `steps` bench steps, over the
+    slowest rank's time (ms)."""
+    return world * units_per_rank_step * steps / (ms_max / 1e3)
+
+
 def max_over_ranks(x: float, world: int, device=None) -> float:
     """Maximum of a per-rank number over all ranks (the job's time is its slowest rank)."""
     if world == 1:
@@ -360,7 +374,7 @@ def run_ours(args):
                         for k in range(K)])
     per_launch_ms = step_ms.mean(axis=0)               # ola_step t, averaged over K
     units_per_step = w.R * w.H * w.B * w.T
-    value = world * units_per_step * K / (ms / 1e3)
+    value = job_value(world, units_per_step, K, ms)
 
     # ---- roofline of the step kernel
     peaks = measured_peaks()

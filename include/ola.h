@@ -203,31 +203,36 @@ ola_status ola_prefill(int32_t R, int32_t H, int32_t d_k, int32_t d_v, int32_t P
                        const float* beta, float* S_out, void* stream);
 
 /* ------------------------------------------------------------------ allocation-free decode
- * Not from the pages: the pages have no counterpart of this entry point. It serves callers
- * that cannot allocate device memory while decoding, e.g. code running inside a CUDA stream
- * capture (a cudaMalloc there breaks the capture), servers whose device memory is fully
- * reserved up front by an arena allocator, and latency-critical loops that cannot afford the
- * implicit synchronisation of an allocation.
+ * Not from the pages: the paper has no counterpart of this entry point. It serves callers that
+ * may not allocate device memory while they decode: servers whose device memory is reserved up
+ * front by an arena or caching allocator (a cudaMalloc behind its back can fail once the arena
+ * holds the device, or fragment it), plugins loaded into a host application that owns every
+ * device allocation, and latency-critical loops that cannot afford the device-wide
+ * synchronisation a cudaMalloc / cudaFree can imply.
  *
  * ola_decode_noalloc runs a whole T_max-step decode of one GDN layer on the fp32 CUDA-core
  * replay path (same results as ola_create + T_max x ola_step + ola_destroy with
  * path = REPLAY, math = FP32), without creating a handle and without allocating anything:
  *   geom        : host pointer; path must be OLA_PATH_REPLAY and math OLA_MATH_FP32; T_max is
- *                 the number of steps decoded; the other limits are those of ola_create.
- *   S_ctx       : device [R][H][d_v][d_k] fp32 shared state (read only).
- *   q, k        : device [T_max][R][B][H][d_k] in_dtype;  v : device [T_max][R][B][H][d_v].
- *   g, beta     : device [T_max][R][B][H] fp32;  parent_idx : device [T_max][R][B] int32.
- *   out_o       : device [T_max][R][B][H][d_v] fp32 (written).
+ *                 the number of steps decoded; the geometry limits are those of ola_create.
+ *   S_ctx       : device [R][H][d_v][d_k] fp32 shared state (read only), 16-byte aligned.
+ *   q, k        : device [T_max][R][B][H][d_k] in_dtype;  v : device [T_max][R][B][H][d_v]
+ *                 (16-byte aligned).
+ *   g, beta     : device [T_max][R][B][H] fp32;  parent_idx : device [T_max][R][B] int32
+ *                 (4-byte aligned); parents as for ola_step, step by step.
+ *   out_o       : device [T_max][R][B][H][d_v] fp32 (written), 16-byte aligned.
  * The transient state (transition records, ancestry rows, error word) lives in one fixed
- * device array of OLA_NOALLOC_SCRATCH_BYTES inside the library, held by every GPU that loads
- * the library until the process exits. Problems needing more than that
- * (ola_noalloc_scratch_bytes) are rejected with OLA_ERR_SCRATCH_LIMIT before anything runs.
- * Every call shares the array and leaves its contents behind; calls whose work overlaps on
- * the GPU (different streams, or several host threads) race on it and must be serialised by
- * the caller. The first call on each device resolves the array's device address (a runtime
- * query, no allocation); make that first call before any stream capture. The call is
- * synchronous: it waits for `stream` and returns the device error status (OLA_OK,
- * OLA_ERR_BAD_PARENT, ...) of this decode. */
+ * device array of OLA_NOALLOC_SCRATCH_BYTES (16 MiB) inside the library, held by every GPU
+ * that loads the library until the process exits. Problems needing more than that
+ * (ola_noalloc_scratch_bytes) are rejected with OLA_ERR_SCRATCH_LIMIT, and bad geometry or
+ * pointers with INVALID_ARG / UNSUPPORTED, before anything is queued. Every call shares the
+ * array and leaves its contents behind (the call clears the error word itself); calls whose
+ * work overlaps on the GPU (different streams, or several host threads) race on it and must be
+ * serialised by the caller. The first call on each device resolves the array's device address
+ * (a runtime query, no allocation); make that first call before any stream capture. The call
+ * is synchronous: it waits for `stream` and returns the device error status (OLA_OK,
+ * OLA_ERR_BAD_PARENT, ...) of this decode; on OLA_ERR_CUDA it has still waited for whatever
+ * it had queued. */
 #define OLA_NOALLOC_SCRATCH_BYTES (16u << 20)
 
 uint64_t ola_noalloc_scratch_bytes(const ola_geometry* geom);

@@ -103,7 +103,12 @@ bool pow2_width(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d =
 bool tc_width(int d) { return d == 64 || d == 128 || d == 256; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-ola_status validate(const ola_geometry* g) {
+}  // namespace
+
+namespace ola {
+
+// Host-side checks of a geometry shared by every entry point that takes one.
+ola_status validate_geometry(const ola_geometry* g) {
   if (!g) return OLA_ERR_INVALID_ARG;
   if (g->R < 1 || g->H < 1 || g->B < 1 || g->T_max < 1) return OLA_ERR_INVALID_ARG;
   if (g->in_dtype != OLA_F32 && g->in_dtype != OLA_BF16) return OLA_ERR_INVALID_ARG;
@@ -120,6 +125,12 @@ ola_status validate(const ola_geometry* g) {
   }
   return OLA_OK;
 }
+
+}  // namespace ola
+
+namespace {
+
+ola_status validate(const ola_geometry* g) { return validate_geometry(g); }
 
 struct Sizes {
   size_t S, S_split, W, Kr, A, C, FS, perm, rank, pchain, err;

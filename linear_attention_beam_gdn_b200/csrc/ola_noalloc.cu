@@ -1,22 +1,24 @@
 // ola_decode_noalloc: a whole T-step decode that allocates no device memory.
 //
-// Who needs this: callers that may not call cudaMalloc at decode time, for example code
-// running while a CUDA stream is being captured into a graph (allocation would break the
-// capture), servers whose device memory is fully pre-reserved by an arena allocator (a
-// cudaMalloc could fail or fragment it), or latency-critical loops where an allocation's
-// implicit synchronisation is not acceptable. They pass every input and output buffer; the
-// transient state of the decode (the transition records, the ancestry rows and the device
-// error word) lives in one fixed array of this file, g_noalloc_scratch, which every GPU that
-// loads the library holds until the process exits.
+// Who needs this: callers that may not call cudaMalloc while they decode. A server whose device
+// memory is reserved up front by an arena or caching allocator cannot let a library take memory
+// behind its back (a cudaMalloc could fail once the arena holds the device, or fragment it); a
+// plugin loaded into a host application may be forbidden to allocate at all; a latency-critical
+// decode loop cannot afford the device-wide synchronisation a cudaMalloc / cudaFree can imply.
+// They pass every input and output buffer; the transient state of the decode (the transition
+// records, the ancestry rows and the device error word) lives in one fixed array of this file,
+// g_noalloc_scratch, which every GPU that loads the library holds until the process exits.
 //
 // The decode runs the CUDA-core fp32 replay kernel (ola_replay_simt.cu) once per step with its
-// record pointers placed inside that array.
+// record pointers placed inside that array. The paper has no counterpart of this entry point.
 #include <mutex>
 
 #include "ola_device.cuh"
 
 namespace ola {
 cudaError_t launch_replay_simt(const StepArgs& a, int in_dtype, cudaStream_t stream);
+size_t replay_simt_smem(int d_k, int d_v, int T_max);
+ola_status validate_geometry(const ola_geometry* g);
 }
 
 using namespace ola;
@@ -32,7 +34,7 @@ std::mutex g_scratch_mutex;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-bool width_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Device address of the scratch array on the current device (resolved once per device).
 cudaError_t scratch_address(unsigned char** out) {
@@ -67,15 +69,30 @@ ola_status ola_decode_noalloc(const ola_geometry* g, const float* S_ctx, const v
                               const void* k, const void* v, const float* gdec,
                               const float* beta, const int32_t* parent_idx, float* out_o,
                               void* stream) {
-  if (!g || !S_ctx || !q || !k || !v || !gdec || !beta || !parent_idx || !out_o)
-    return OLA_ERR_INVALID_ARG;
-  if (g->R < 1 || g->H < 1 || g->B < 1 || g->T_max < 1) return OLA_ERR_INVALID_ARG;
-  if (g->in_dtype != OLA_F32 && g->in_dtype != OLA_BF16) return OLA_ERR_INVALID_ARG;
+  // host-side checks first (no CUDA call before they pass): the geometry limits of ola_create
+  // and the pointer rules of ola_create / ola_step
+  ola_status vs = validate_geometry(g);
+  if (vs != OLA_OK) return vs;
   if (g->path != OLA_PATH_REPLAY || g->math != OLA_MATH_FP32) return OLA_ERR_UNSUPPORTED;
-  if (!width_ok(g->d_k) || !width_ok(g->d_v) || g->B > 4096 || g->T_max > 32)
-    return OLA_ERR_UNSUPPORTED;
+  if (!S_ctx || !q || !k || !v || !gdec || !beta || !parent_idx || !out_o)
+    return OLA_ERR_INVALID_ARG;
+  if (!aligned(S_ctx, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+      !aligned(out_o, 16) || !aligned(gdec, 4) || !aligned(beta, 4) || !aligned(parent_idx, 4))
+    return OLA_ERR_INVALID_ARG;
   const uint64_t need = ola_noalloc_scratch_bytes(g);
   if (need > OLA_NOALLOC_SCRATCH_BYTES) return OLA_ERR_SCRATCH_LIMIT;
+  // device checks (attribute queries only): an sm_100 device whose shared memory holds the
+  // kernel's per-block footprint
+  int dev = 0, major = 0, smem_optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return OLA_ERR_CUDA;
+  }
+  if (major != 10 || replay_simt_smem(g->d_k, g->d_v, g->T_max) > size_t(smem_optin))
+    return OLA_ERR_UNSUPPORTED;
 
   unsigned char* base = nullptr;
   cudaError_t e = scratch_address(&base);
@@ -125,6 +142,10 @@ ola_status ola_decode_noalloc(const ola_geometry* g, const float* S_ctx, const v
   if (e == cudaSuccess) e = cudaMemcpyAsync(word, err, 16, cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) {
+    // a launch that failed part-way leaves the earlier steps queued: wait for them, so that
+    // no kernel of this call still writes the scratch array once the call has returned
+    cudaGetLastError();
+    cudaStreamSynchronize(st);
     cudaGetLastError();
     return OLA_ERR_CUDA;
   }

@@ -226,11 +226,6 @@ def closed_form_state(S_ctx: np.ndarray, records: list, chain: Sequence[int]) ->
 
 # ----------------------------------------------------------------------------- batched layouts
 
-def decode_unit(S_ctx_rh, steps_q, steps_k, steps_v, steps_g, steps_beta, parents_r):
-    """One (request, head) unit in the library's layout slices; arrays already fp64."""
-    return full_state_decode(S_ctx_rh, steps_q, steps_k, steps_v, steps_g, steps_beta, parents_r)
-
-
 def decode_batch(S_ctx: np.ndarray, q: np.ndarray, k: np.ndarray, v: np.ndarray, g: np.ndarray,
                  beta: np.ndarray, parents: np.ndarray, units=None) -> np.ndarray:
     """Oracle over the library's tensor layout.

@@ -1,9 +1,12 @@
 """The multi-rank path on the CPU: world_size-2 `gloo` process groups.
 
-Requests are independent, so ranks split them with no collective on the data path: each rank
-decodes its own requests (here with the oracle, on the CPU) and only the timing is reduced
-(max over ranks). These tests check the request sharding, that the per-rank results put
-together equal the single-process decode, and the max-over-ranks reduction bench.py uses."""
+Requests are independent, so bench.py gives every rank its own batch of requests (the same
+shape, its own seeds: bench.rank_workload) with no collective on the data path; only the timing
+is reduced (bench.max_over_ranks) and the job's value is every rank's units over the slowest
+rank's time (bench.job_value). These tests run that rank logic in two gloo ranks, each decoding
+its own batch with the oracle on the CPU, and check that every rank's result equals the
+single-process decode of that rank's workload, that the ranks' batches differ, and the
+max-over-ranks reduction and job value."""
 import os
 import socket
 
@@ -17,6 +20,8 @@ import bench
 import oracle
 import workloads as wl
 
+BASE = dict(R=2, P=16)
+
 
 def _free_port():
     s = socket.socket()
@@ -26,19 +31,17 @@ def _free_port():
     return port
 
 
-def _decode_requests(w, lo, hi):
+def _decode_all(w):
     steps = wl.make_all_steps(w)
     par = wl.make_parents(w)
     prompt = wl.make_prompt(w, "cpu")
     f = lambda key: np.stack([oracle.as_f64(s[key]) for s in steps])
     S = np.zeros((w.R, w.H, w.d_v, w.d_k))
-    for r in range(lo, hi):
+    for r in range(w.R):
         for h in range(w.H):
             S[r, h] = oracle.prefill(*(oracle.as_f64(prompt[x][r, :, h])
                                        for x in ("k", "v", "g", "beta")))
-    units = [(r, h) for r in range(lo, hi) for h in range(w.H)]
-    o = oracle.decode_batch(S, f("q"), f("k"), f("v"), f("g"), f("beta"), par, units=units)
-    return o[:, lo:hi]
+    return oracle.decode_batch(S, f("q"), f("k"), f("v"), f("g"), f("beta"), par)
 
 
 def _worker(rank, world, port, result_q):
@@ -46,20 +49,21 @@ def _worker(rank, world, port, result_q):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=__import__("datetime").timedelta(seconds=60))
     try:
-        w = wl.WORKLOADS["tiny"].scaled(R=5, P=16)
-        lo, hi = wl.shard_requests(w.R, world, rank)
-        part = _decode_requests(w, lo, hi)
+        w = bench.rank_workload(wl.WORKLOADS["tiny"].scaled(**BASE), rank)
+        part = _decode_all(w)
         parts = [None] * world
-        dist.all_gather_object(parts, (lo, hi, part))
-        slowest = bench.max_over_ranks(float(rank + 1) * 1.5, world)
+        dist.all_gather_object(parts, (rank, w.seed, part))
+        ms = float(rank + 1) * 1.5
+        slowest = bench.max_over_ranks(ms, world)
+        value = bench.job_value(world, w.R * w.H * w.B * w.T, 4, slowest)
         if rank == 0:
-            result_q.put((parts, slowest))
+            result_q.put((parts, slowest, value))
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
-def test_two_ranks_shard_requests_and_reduce_time():
+def test_two_ranks_decode_their_own_batches_and_reduce_time():
     world = 2
     port = _free_port()
     ctx = tmp.get_context("spawn")
@@ -67,18 +71,22 @@ def test_two_ranks_shard_requests_and_reduce_time():
     procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
-    parts, slowest = q.get(timeout=240)
+    parts, slowest, value = q.get(timeout=240)
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
     assert slowest == 3.0
+    base = wl.WORKLOADS["tiny"].scaled(**BASE)
+    units = base.R * base.H * base.B * base.T
+    assert value == pytest.approx(2 * units * 4 / 3.0e-3)
     parts = sorted(parts, key=lambda x: x[0])
-    assert parts[0][0] == 0 and parts[-1][1] == 5
-    assert all(a[1] == b[0] for a, b in zip(parts, parts[1:]))
-    joined = np.concatenate([p[2] for p in parts], axis=1)
-    w = wl.WORKLOADS["tiny"].scaled(R=5, P=16)
-    whole = _decode_requests(w, 0, w.R)
-    np.testing.assert_array_equal(joined, whole)
+    assert [p[0] for p in parts] == [0, 1]
+    assert parts[0][1] != parts[1][1]                       # distinct seeds
+    assert not np.allclose(parts[0][2], parts[1][2])         # distinct batches
+    for rank, seed, o in parts:
+        w = bench.rank_workload(base, rank)
+        assert w.seed == seed
+        np.testing.assert_array_equal(o, _decode_all(w))
 
 
 def test_rank_workloads_are_distinct():

@@ -83,3 +83,39 @@ def test_pins_reject_mutant(name, monkeypatch):
 
 def test_pins_accept_original():
     assert not _golden_fails() and not _property_fails()
+
+
+def _ancestry_mutants():
+    original = gdn_oracle.ancestry_table
+
+    def first_request_only(parents):        # every request takes request 0's parents
+        T, R, B = parents.shape
+        out = np.zeros((R, B, T), dtype=np.int32)
+        for r in range(R):
+            out[r] = np.array(gdn_oracle.chains(parents[:, 0])[T - 1], dtype=np.int32)
+        return out
+
+    def slots_reversed(parents):             # newest record first
+        return original(parents)[:, :, ::-1]
+
+    def own_index_everywhere(parents):       # beam b at every slot: parents never followed
+        T, R, B = parents.shape
+        out = np.zeros((R, B, T), dtype=np.int32)
+        out[:] = np.arange(B, dtype=np.int32)[None, :, None]
+        return out
+
+    return {"first_request_only": first_request_only, "slots_reversed": slots_reversed,
+            "own_index_everywhere": own_index_everywhere}
+
+
+@pytest.mark.parametrize("name", list(_ancestry_mutants()))
+def test_ancestry_pin_rejects_mutant(name, monkeypatch):
+    import test_oracle_pins as pins
+    monkeypatch.setattr(oracle, "ancestry_table", _ancestry_mutants()[name])
+    with pytest.raises(AssertionError):
+        pins.test_ancestry_table_by_walking_parent_pointers()
+
+
+def test_ancestry_pin_accepts_original():
+    import test_oracle_pins as pins
+    pins.test_ancestry_table_by_walking_parent_pointers()

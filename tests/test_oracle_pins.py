@@ -274,9 +274,41 @@ def test_chains_by_walking_parent_pointers():
                 assert ch[t][b][t] == b
                 if t > 0:
                     assert ch[t][b][:t] == ch[t - 1][par[t, r, b]]
+
+
+def _walk_table(par):
+    """[R, B, T] record beam index of every slot of every final beam, by climbing the parent
+    pointers from (T-1, b) of each request to the root."""
+    T, R, B = par.shape
+    out = np.zeros((R, B, T), dtype=np.int64)
+    for r in range(R):
+        for b in range(B):
+            cur = b
+            for s in range(T - 1, -1, -1):
+                out[r, b, s] = cur
+                cur = par[s, r, cur]
+    return out
+
+
+def test_ancestry_table_by_walking_parent_pointers():
+    """Every entry of the table, for every request: requests draw different parents (their
+    own seeds), so a table built from one request's parents for all of them fails."""
+    W = wl.WORKLOADS["stress"].scaled(R=3, B=48, T=5, max_children=6)
+    par = wl.make_parents(W)
+    assert not np.array_equal(par[:, 0], par[:, 1]) and not np.array_equal(par[:, 1], par[:, 2])
     table = oracle.ancestry_table(par)
     assert table.shape == (W.R, W.B, W.T)
-    assert np.array_equal(table[:, :, -1], np.tile(np.arange(W.B), (W.R, 1)))
+    assert np.array_equal(table, _walk_table(par))
+    # a hand-made two-request tree: request 0 keeps every beam, request 1 follows beam 1
+    par2 = np.zeros((3, 2, 3), dtype=np.int32)
+    par2[1, 0] = [0, 1, 2]
+    par2[2, 0] = [2, 0, 1]
+    par2[1, 1] = [1, 1, 0]
+    par2[2, 1] = [1, 2, 2]
+    # worked by hand: slot s of final beam b is the beam it descends from at step s
+    exp = np.array([[[2, 2, 0], [0, 0, 1], [1, 1, 2]],
+                    [[1, 1, 0], [0, 2, 1], [0, 2, 2]]])
+    assert np.array_equal(oracle.ancestry_table(par2), exp)
 
 
 def test_bad_parents_rejected():

@@ -202,14 +202,6 @@ def make_all_steps(w: Workload, device="cpu") -> List[Dict[str, torch.Tensor]]:
     return [make_step_inputs(w, t, device) for t in range(w.T)]
 
 
-def shard_requests(R: int, world: int, rank: int) -> Tuple[int, int]:
-    """Contiguous block of requests [lo, hi) owned by `rank` out of `world` ranks."""
-    base, rem = divmod(R, world)
-    lo = rank * base + min(rank, rem)
-    hi = lo + base + (1 if rank < rem else 0)
-    return lo, hi
-
-
 def distinct_ancestor_counts(parents: np.ndarray) -> np.ndarray:
     """U[t][r]: number of distinct (step, beam) records at steps < t reachable from the beams
     of step t through the parent tables (pure bookkeeping on integer parent tables, used to
