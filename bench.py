@@ -413,7 +413,8 @@ def run_ours(args):
     comps = {}
     if not args.no_compare:
         for name, p, m, reps in (("replay_fp32", ola.OLA_PATH_REPLAY, ola.OLA_MATH_FP32, 2),
-                                 ("fullstate", ola.OLA_PATH_FULLSTATE, ola.OLA_MATH_FP32, 2)):
+                                 ("fullstate", ola.OLA_PATH_FULLSTATE, ola.OLA_MATH_FP32, 2),
+                                 ("replayssm", ola.OLA_PATH_REPLAYSSM, ola.OLA_MATH_FP32, 2)):
             try:
                 d2 = ola.Decoder(S, B=w.B, T_max=w.T, in_dtype=w.torch_dtype, path=p, math=m)
             except ola.OlaError as ex:

@@ -64,8 +64,14 @@ typedef enum {
 
 /* dtype of q, k, v (and of the prompt's k, v for ola_prefill) */
 enum { OLA_F32 = 0, OLA_BF16 = 1 };
-/* how beam states are represented */
-enum { OLA_PATH_REPLAY = 0, OLA_PATH_FULLSTATE = 1 };
+/* how beam states are represented:
+ * REPLAY     = one shared state + append-only transition records (w, k, alpha) per beam,
+ *              evaluated by projection replay (the method);
+ * FULLSTATE  = one materialised d_v x d_k fp32 state per beam, ping-pong buffers (comparison);
+ * REPLAYSSM  = no per-beam state kept: each step rebuilds every beam's state from the shared
+ *              state by replaying the raw tokens (k, v, alpha, beta) on its chain, fp32
+ *              (comparison). */
+enum { OLA_PATH_REPLAY = 0, OLA_PATH_FULLSTATE = 1, OLA_PATH_REPLAYSSM = 2 };
 /* how the contractions of the replay path are computed:
  * FP32 = CUDA-core fp32 FMA everywhere; TENSOR = tcgen05 tensor cores, bf16 operands with
  * S_ctx split into a bf16 high part and a bf16 remainder (two MMAs, fp32 accumulate in
@@ -83,7 +89,7 @@ typedef struct {
   int32_t B;          /* beams per request, 1..4096 (TENSOR: T_max*R*H*B < 2^31) */
   int32_t T_max;      /* decode steps the handle can hold, 1..32 */
   int32_t in_dtype;   /* OLA_F32 or OLA_BF16 (TENSOR: OLA_BF16) */
-  int32_t path;       /* OLA_PATH_REPLAY or OLA_PATH_FULLSTATE */
+  int32_t path;       /* OLA_PATH_REPLAY, OLA_PATH_FULLSTATE or OLA_PATH_REPLAYSSM */
   int32_t math;       /* OLA_MATH_FP32 or OLA_MATH_TENSOR (replay path only) */
 } ola_geometry;
 
@@ -174,7 +180,8 @@ ola_status ola_get_error(ola_handle h);
  * ranks down by that many slots and decreases t by it. Later steps give the same outputs up to
  * rounding, and a decode can run past T_max while its beams keep converging. The current
  * step's own records are never folded (t stays >= 1). ola_get_ancestry afterwards returns the
- * chains without the folded slots, and ola_reset keeps the folded S_ctx.
+ * chains without the folded slots, and ola_reset keeps the folded S_ctx. On the REPLAYSSM
+ * path the folded records are raw tokens and are applied with the gated delta rule itself.
  *   out_folded : host int32, optional (NULL): number of folded steps (0 if none).
  * Synchronises `stream`, which must be the stream of the handle's previous calls (or ordered
  * after them). FullState handles hold no records: nothing is folded.

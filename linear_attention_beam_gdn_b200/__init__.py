@@ -16,7 +16,8 @@ import re
 from typing import Optional
 
 __all__ = ["OlaError", "LibraryMissing", "Geometry", "lib", "Decoder", "prefill",
-           "OLA_F32", "OLA_BF16", "OLA_PATH_REPLAY", "OLA_PATH_FULLSTATE", "OLA_MATH_FP32",
+           "OLA_F32", "OLA_BF16", "OLA_PATH_REPLAY", "OLA_PATH_FULLSTATE", "OLA_PATH_REPLAYSSM",
+           "OLA_MATH_FP32",
            "OLA_MATH_TENSOR", "LIB_PATH", "HEADER_PATH", "declared_symbols"]
 
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -28,7 +29,7 @@ OLA_ERR_BAD_PARENT, OLA_ERR_OOM, OLA_ERR_CUDA, OLA_ERR_TIMEOUT = 4, 5, 6, 7
 OLA_ERR_SCRATCH_LIMIT = 8
 OLA_NOALLOC_SCRATCH_BYTES = 16 << 20
 OLA_F32, OLA_BF16 = 0, 1
-OLA_PATH_REPLAY, OLA_PATH_FULLSTATE = 0, 1
+OLA_PATH_REPLAY, OLA_PATH_FULLSTATE, OLA_PATH_REPLAYSSM = 0, 1, 2
 OLA_MATH_FP32, OLA_MATH_TENSOR = 0, 1
 
 

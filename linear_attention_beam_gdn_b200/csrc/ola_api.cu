@@ -20,6 +20,7 @@ cudaError_t launch_prefill_chunk(int R, int H, int P, const void* k, const void*
                                  const float* g, const float* beta, float* S_out, int* err,
                                  cudaStream_t stream);
 cudaError_t launch_fullstate(const StepArgs& a, int in_dtype, cudaStream_t stream);
+cudaError_t launch_replayssm(const StepArgs& a, int in_dtype, cudaStream_t stream);
 cudaError_t launch_replay_simt(const StepArgs& a, int in_dtype, cudaStream_t stream);
 size_t replay_simt_smem(int d_k, int d_v, int T_max);
 cudaError_t launch_replay_tc(const StepArgs& a, const CUtensorMap& mhi, const CUtensorMap& mlo,
@@ -35,7 +36,7 @@ size_t replay_pipe_smem(int d_k, int T_max);
 cudaError_t launch_replay_pipe(const StepArgs& a, const void* S_hi, const void* S_lo,
                                cudaStream_t stream);
 bool replay_mma_supported(int d_k, int d_v, int B, int T_max);
-size_t replay_mma_smem(int d_k);
+size_t replay_mma_smem(int d_k, int d_v);
 size_t plan_units_smem(int B, int T_max);
 cudaError_t launch_replay_mma(const StepArgs& a, const UnitPlan& up, const void* S_hi,
                               const void* S_lo, const CUtensorMap& mkr, const CUtensorMap& mw,
@@ -47,8 +48,8 @@ cudaError_t launch_split_state(const float* S, void* hi, void* lo, int RH, int d
 cudaError_t launch_common_prefix(const int* C, int R, int B, int T_max, int t, int* out,
                                  cudaStream_t stream);
 cudaError_t launch_fold(float* S, const void* W, const void* Kr, int k_is_bf16, const float* A,
-                        const int* C, int R, int H, int d_k, int d_v, int B, int T_max, int t,
-                        int c, int layout, cudaStream_t stream);
+                        const float* Bt, const int* C, int R, int H, int d_k, int d_v, int B,
+                        int T_max, int t, int c, int layout, cudaStream_t stream);
 cudaError_t launch_chain_shift(int* C, int R, int B, int T_max, int t, int c, cudaStream_t stream);
 }  // namespace ola
 
@@ -65,6 +66,8 @@ struct ola_ctx {
   float* W = nullptr;
   void* Kr = nullptr;
   float* A = nullptr;
+  void* Vr = nullptr;        // history-replay path: v of every record
+  float* Br = nullptr;       // history-replay path: beta of every record
   int* C = nullptr;
   float* FS[2] = {nullptr, nullptr};
   int* perm = nullptr;       // [2][R][B] depth-first order of the current step and the
@@ -72,6 +75,7 @@ struct ola_ctx {
   int* rank = nullptr;       // [2][R][B] depth-first position of each beam, by step parity
   int* pchain = nullptr;     // [R][B][T_max] parent chain by depth-first position
   int* err = nullptr;
+  int* lens = nullptr;       // [R] shared chain prefix of each request (ola_compact)
   CUtensorMap m_hi, m_lo;
   CUtensorMap m_kr, m_w;     // record row maps of the mma kernel
   bool pipe = false;         // tensor path on the persistent pipelined kernel
@@ -112,7 +116,9 @@ ola_status validate_geometry(const ola_geometry* g) {
   if (!g) return OLA_ERR_INVALID_ARG;
   if (g->R < 1 || g->H < 1 || g->B < 1 || g->T_max < 1) return OLA_ERR_INVALID_ARG;
   if (g->in_dtype != OLA_F32 && g->in_dtype != OLA_BF16) return OLA_ERR_INVALID_ARG;
-  if (g->path != OLA_PATH_REPLAY && g->path != OLA_PATH_FULLSTATE) return OLA_ERR_INVALID_ARG;
+  if (g->path != OLA_PATH_REPLAY && g->path != OLA_PATH_FULLSTATE &&
+      g->path != OLA_PATH_REPLAYSSM)
+    return OLA_ERR_INVALID_ARG;
   if (g->math != OLA_MATH_FP32 && g->math != OLA_MATH_TENSOR) return OLA_ERR_INVALID_ARG;
   if (!pow2_width(g->d_k) || !pow2_width(g->d_v)) return OLA_ERR_UNSUPPORTED;
   if (g->B > 4096 || g->T_max > 32) return OLA_ERR_UNSUPPORTED;
@@ -133,11 +139,11 @@ namespace {
 ola_status validate(const ola_geometry* g) { return validate_geometry(g); }
 
 struct Sizes {
-  size_t S, S_split, W, Kr, A, C, FS, perm, rank, pchain, err;
+  size_t S, S_split, W, Kr, A, Vr, Br, C, FS, perm, rank, pchain, err, lens;
   size_t ucnt, uoff, urec, upos, counter;   // mma path only
   size_t total() const {
-    return S + 2 * S_split + W + Kr + A + C + 2 * FS + perm + rank + pchain + err + ucnt + uoff +
-           urec + upos + counter;
+    return S + 2 * S_split + W + Kr + A + Vr + Br + C + 2 * FS + perm + rank + pchain + err +
+           lens + ucnt + uoff + urec + upos + counter;
   }
 };
 
@@ -152,16 +158,19 @@ Sizes sizes_of(const ola_geometry* g) {
   const size_t e = g->in_dtype == OLA_BF16 ? 2 : 4;
   z.S = R * H * dv * dk * 4;
   z.S_split = g->math == OLA_MATH_TENSOR ? R * H * ((dv + 127) / 128 * 128) * dk * 2 : 0;
-  const bool rep = g->path == OLA_PATH_REPLAY;
+  const bool rep = g->path == OLA_PATH_REPLAY, rss = g->path == OLA_PATH_REPLAYSSM;
   z.W = rep ? T * R * H * B * dv * 4 : 0;
-  z.Kr = rep ? T * R * H * B * dk * e : 0;
-  z.A = rep ? T * R * H * B * 4 : 0;
+  z.Kr = rep ? T * R * H * B * dk * e : rss ? T * R * H * B * dk * 4 : 0;
+  z.A = (rep || rss) ? T * R * H * B * 4 : 0;
+  z.Vr = rss ? T * R * H * B * dv * 4 : 0;
+  z.Br = rss ? T * R * H * B * 4 : 0;
   z.C = T * R * B * T * 4;
-  z.FS = rep ? 0 : R * H * B * dv * dk * 4;
+  z.FS = g->path == OLA_PATH_FULLSTATE ? R * H * B * dv * dk * 4 : 0;
   z.perm = g->math == OLA_MATH_TENSOR ? 2 * R * B * 4 : 0;
   z.rank = g->math == OLA_MATH_TENSOR ? 2 * R * B * 4 : 0;
   z.pchain = g->math == OLA_MATH_TENSOR ? R * B * T * 4 : 0;
   z.err = 16;
+  z.lens = g->path != OLA_PATH_FULLSTATE ? R * 4 : 0;
   if (uses_mma(g)) {
     z.ucnt = R * 4;
     z.uoff = (R + 1) * 4;
@@ -190,9 +199,10 @@ cudaError_t dev_alloc(T** p, size_t bytes) {
 }
 
 void free_all(ola_ctx* h) {
-  void* ptrs[] = {h->S,     h->S_hi,  h->S_lo,   h->W,       h->Kr,     h->A,
+  void* ptrs[] = {h->S,     h->S_hi,  h->S_lo,   h->W,       h->Kr,     h->A,  h->Vr, h->Br,
                   h->C,     h->FS[0], h->FS[1],  h->perm,    h->rank,   h->pchain,
-                  h->err,   h->up.ucnt, h->up.uoff, h->up.urec, h->up.upos, h->up.counter};
+                  h->err,   h->lens,  h->up.ucnt, h->up.uoff, h->up.urec, h->up.upos,
+                  h->up.counter};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (void* p : h->st)
@@ -240,6 +250,8 @@ StepArgs make_args(ola_ctx* h, const void* q, const void* k, const void* v, cons
   a.rank_prev = h->rank ? h->rank + ((a.t + 1) & 1) * RB : nullptr;
   a.rank_cur = h->rank ? h->rank + (a.t & 1) * RB : nullptr;
   a.err = h->err;
+  a.Vr = h->Vr;
+  a.Br = h->Br;
   return a;
 }
 
@@ -287,7 +299,7 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
   if (geom->path == OLA_PATH_REPLAY) {
     size_t smem = geom->math != OLA_MATH_TENSOR
                       ? replay_simt_smem(geom->d_k, geom->d_v, geom->T_max)
-                  : uses_mma(geom) ? replay_mma_smem(geom->d_k)
+                  : uses_mma(geom) ? replay_mma_smem(geom->d_k, geom->d_v)
                   : replay_pipe_supported(geom->d_k, geom->d_v, geom->T_max)
                       ? replay_pipe_smem(geom->d_k, geom->T_max)
                   : replay_pos_supported(geom->d_k, geom->d_v)
@@ -315,6 +327,8 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
   if (e == cudaSuccess) e = dev_alloc(&h->W, z.W);
   if (e == cudaSuccess) e = dev_alloc(&h->Kr, z.Kr);
   if (e == cudaSuccess) e = dev_alloc(&h->A, z.A);
+  if (e == cudaSuccess) e = dev_alloc(&h->Vr, z.Vr);
+  if (e == cudaSuccess) e = dev_alloc(&h->Br, z.Br);
   if (e == cudaSuccess) e = dev_alloc(&h->C, z.C);
   if (e == cudaSuccess) e = dev_alloc(&h->FS[0], z.FS);
   if (e == cudaSuccess) e = dev_alloc(&h->FS[1], z.FS);
@@ -322,6 +336,7 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
   if (e == cudaSuccess) e = dev_alloc(&h->rank, z.rank);
   if (e == cudaSuccess) e = dev_alloc(&h->pchain, z.pchain);
   if (e == cudaSuccess) e = dev_alloc(&h->err, z.err);
+  if (e == cudaSuccess) e = dev_alloc(&h->lens, z.lens);
   if (e == cudaSuccess) e = dev_alloc(&h->up.ucnt, z.ucnt);
   if (e == cudaSuccess) e = dev_alloc(&h->up.uoff, z.uoff);
   if (e == cudaSuccess) e = dev_alloc(&h->up.urec, z.urec);
@@ -370,6 +385,8 @@ ola_status ola_step(ola_handle h, const void* q, const void* k, const void* v, c
   cudaError_t e;
   if (h->g.path == OLA_PATH_FULLSTATE)
     e = launch_fullstate(a, h->g.in_dtype, st);
+  else if (h->g.path == OLA_PATH_REPLAYSSM)
+    e = launch_replayssm(a, h->g.in_dtype, st);
   else if (h->g.math == OLA_MATH_TENSOR && h->mma)
     e = launch_replay_mma(a, h->up, h->S_hi, h->S_lo, h->m_kr, h->m_w, st);
   else if (h->g.math == OLA_MATH_TENSOR && h->pipe)
@@ -497,14 +514,11 @@ ola_status ola_compact(ola_handle h, int32_t* out_folded, void* stream) {
   if (g.path == OLA_PATH_FULLSTATE || t < 2) return OLA_OK;   // nothing to fold
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;
-  // shared chain prefix of every request
-  int* lens = nullptr;
-  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&lens), size_t(g.R) * 4, st);
-  if (e == cudaSuccess) e = launch_common_prefix(h->C, g.R, g.B, g.T_max, t, lens, st);
+  // shared chain prefix of every request (into the handle's own buffer: nothing is allocated)
+  cudaError_t e = launch_common_prefix(h->C, g.R, g.B, g.T_max, t, h->lens, st);
   std::vector<int> host(size_t(g.R), 0);
   if (e == cudaSuccess)
-    e = cudaMemcpyAsync(host.data(), lens, size_t(g.R) * 4, cudaMemcpyDeviceToHost, st);
-  if (lens) cudaFreeAsync(lens, st);
+    e = cudaMemcpyAsync(host.data(), h->lens, size_t(g.R) * 4, cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return from_cuda(e);
   int c = t - 1;
@@ -512,24 +526,25 @@ ola_status ola_compact(ola_handle h, int32_t* out_folded, void* stream) {
   if (c <= 0) return OLA_OK;
   // fold the shared records into S_ctx (and its bf16 split), then move the later record slots
   // and the chain rows down by c
-  const int layout = h->mma ? 1 : 0;
-  e = launch_fold(h->S, h->W, h->Kr, g.in_dtype == OLA_BF16, h->A, h->C, g.R, g.H, g.d_k, g.d_v,
-                  g.B, g.T_max, t, c, layout, st);
+  const bool rss = g.path == OLA_PATH_REPLAYSSM;
+  const int layout = rss ? 2 : h->mma ? 1 : 0;
+  e = launch_fold(h->S, rss ? h->Vr : h->W, h->Kr, !rss && g.in_dtype == OLA_BF16, h->A, h->Br,
+                  h->C, g.R, g.H, g.d_k, g.d_v, g.B, g.T_max, t, c, layout, st);
   if (e == cudaSuccess && g.math == OLA_MATH_TENSOR)
     e = launch_split_state(h->S, h->S_hi, h->S_lo, g.R * g.H, g.d_k, g.d_v, st);
   const size_t rows = size_t(g.R) * g.H * g.B;
   const size_t kbytes = g.in_dtype == OLA_BF16 ? 2 : 4;
-  const size_t w_slot = rows * g.d_v * 4, k_slot = rows * g.d_k * kbytes, a_slot = rows * 4;
-  for (int s = c; s < t && e == cudaSuccess; ++s) {   // increasing order: sources stay intact
-    char* W = reinterpret_cast<char*>(h->W);
-    char* K = static_cast<char*>(h->Kr);
-    char* A = reinterpret_cast<char*>(h->A);
-    e = cudaMemcpyAsync(W + (s - c) * w_slot, W + s * w_slot, w_slot, cudaMemcpyDeviceToDevice, st);
-    if (e == cudaSuccess)
-      e = cudaMemcpyAsync(K + (s - c) * k_slot, K + s * k_slot, k_slot, cudaMemcpyDeviceToDevice, st);
-    if (e == cudaSuccess)
-      e = cudaMemcpyAsync(A + (s - c) * a_slot, A + s * a_slot, a_slot, cudaMemcpyDeviceToDevice, st);
-  }
+  // per record slot: w (or, on the history-replay path, v and beta), k, alpha
+  const size_t w_slot = rows * g.d_v * 4;
+  const size_t k_slot = rows * g.d_k * (rss ? 4 : kbytes), a_slot = rows * 4;
+  char* const bufs[4] = {reinterpret_cast<char*>(rss ? h->Vr : h->W), static_cast<char*>(h->Kr),
+                         reinterpret_cast<char*>(h->A), reinterpret_cast<char*>(h->Br)};
+  const size_t slot_bytes[4] = {w_slot, k_slot, a_slot, rss ? a_slot : 0};
+  for (int s = c; s < t && e == cudaSuccess; ++s)     // increasing order: sources stay intact
+    for (int x = 0; x < 4 && e == cudaSuccess; ++x)
+      if (slot_bytes[x])
+        e = cudaMemcpyAsync(bufs[x] + (s - c) * slot_bytes[x], bufs[x] + s * slot_bytes[x],
+                            slot_bytes[x], cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = launch_chain_shift(h->C, g.R, g.B, g.T_max, t, c, st);
   // the next step reads the depth-first ranks of this one from the buffer of its parity
   const size_t RB = size_t(g.R) * g.B;

@@ -44,10 +44,14 @@ __global__ void __launch_bounds__(256) common_prefix_kernel(const int* __restric
 // chain: every beam shares them). One thread per state row.
 //   layout 0: records [T_max][R][H][B], w fp32 [d_v]
 //   layout 1: records [T_max][R][B][H], w as bf16 hi and lo planes [2][d_v]
+//   layout 2: records [T_max][R][H][B] holding the raw token (history-replay path): k and v
+//             in fp32, and beta; w_j[i] = beta_j (v_j[i] - alpha_j S_i . k_j) is formed
+//             from the state folded so far (the gated delta rule itself)
 template <typename TK>
 __global__ void __launch_bounds__(128) fold_kernel(float* __restrict__ S, const void* __restrict__ Wp,
                                                   const TK* __restrict__ Kr,
                                                   const float* __restrict__ A,
+                                                  const float* __restrict__ Bt,
                                                   const int* __restrict__ C, int R, int H,
                                                   int d_k, int d_v, int B, int T_max, int t,
                                                   int c, int layout) {
@@ -60,17 +64,21 @@ __global__ void __launch_bounds__(128) fold_kernel(float* __restrict__ S, const 
   const int* chain = C + (size_t(t - 1) * R + r) * size_t(B) * T_max;   // beam 0's chain
   for (int s = 0; s < c; ++s) {
     const int b = chain[s];
-    const size_t rec = layout == 0 ? ((size_t(s) * R + r) * H + h) * size_t(B) + b
+    const size_t rec = layout != 1 ? ((size_t(s) * R + r) * H + h) * size_t(B) + b
                                    : ((size_t(s) * R + r) * B + b) * size_t(H) + h;
+    const float al = A[rec];
+    const TK* k = Kr + rec * d_k;
     float w;
     if (layout == 0) {
       w = static_cast<const float*>(Wp)[rec * d_v + i];
-    } else {
+    } else if (layout == 1) {
       const __nv_bfloat16* wb = static_cast<const __nv_bfloat16*>(Wp) + rec * 2 * d_v;
       w = __bfloat162float(wb[i]) + __bfloat162float(wb[d_v + i]);
+    } else {
+      float u = 0.f;
+      for (int x = 0; x < d_k; ++x) u = fmaf(Srow[x], float(k[x]), u);
+      w = Bt[rec] * (float(static_cast<const TK*>(Wp)[rec * d_v + i]) - al * u);
     }
-    const float al = A[rec];
-    const TK* k = Kr + rec * d_k;
     for (int x = 0; x < d_k; ++x) Srow[x] = fmaf(al, Srow[x], w * float(k[x]));
   }
 }
@@ -91,16 +99,17 @@ cudaError_t launch_common_prefix(const int* C, int R, int B, int T_max, int t, i
 }
 
 cudaError_t launch_fold(float* S, const void* W, const void* Kr, int k_is_bf16, const float* A,
-                        const int* C, int R, int H, int d_k, int d_v, int B, int T_max, int t,
-                        int c, int layout, cudaStream_t stream) {
+                        const float* Bt, const int* C, int R, int H, int d_k, int d_v, int B,
+                        int T_max, int t, int c, int layout, cudaStream_t stream) {
   const size_t rows = size_t(R) * H * d_v;
   const unsigned grid = unsigned((rows + 127) / 128);
   if (k_is_bf16)
     fold_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>(
-        S, W, static_cast<const __nv_bfloat16*>(Kr), A, C, R, H, d_k, d_v, B, T_max, t, c, layout);
+        S, W, static_cast<const __nv_bfloat16*>(Kr), A, Bt, C, R, H, d_k, d_v, B, T_max, t, c,
+        layout);
   else
-    fold_kernel<float><<<grid, 128, 0, stream>>>(S, W, static_cast<const float*>(Kr), A, C, R, H,
-                                                 d_k, d_v, B, T_max, t, c, layout);
+    fold_kernel<float><<<grid, 128, 0, stream>>>(S, W, static_cast<const float*>(Kr), A, Bt, C, R,
+                                                 H, d_k, d_v, B, T_max, t, c, layout);
   return cudaGetLastError();
 }
 

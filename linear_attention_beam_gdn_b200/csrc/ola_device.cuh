@@ -13,7 +13,7 @@
 namespace ola {
 
 // Everything one decode step needs. Record storage (the transition records of every beam,
-// appended once and never moved):
+// appended once and never moved; the history-replay path keeps v_t and beta_t instead of w_t):
 //   W  [T_max][R][H][B][d_v] fp32   w_t = beta (v - alpha u)
 //   Kr [T_max][R][H][B][d_k] in_dtype  copy of k_t
 //   A  [T_max][R][H][B]      fp32   alpha_t = exp(g_t)
@@ -43,6 +43,9 @@ struct StepArgs {
   const int* rank_prev;         // [R][B] depth-first position of each beam of step t-1
   int* rank_cur;                // [R][B] depth-first position of each beam of step t
   int* err;                     // device error word: [0] code, [1] detail, [2] step
+  // history-replay path only: the raw tokens of every step (Kr holds the keys, in fp32)
+  void* Vr;                     // [T_max][R][H][B][d_v] fp32      v_t
+  float* Br;                    // [T_max][R][H][B]      fp32      beta_t
 };
 
 // Units of work of the tensor-core replay kernel, written each step by plan_units_kernel

@@ -1,5 +1,5 @@
 // Projection-replay decode step with both contractions on tensor cores: persistent, pipelined,
-// state-major (sm_100a; d_v = 128, d_k = 64 or 128, T_max <= 12, B <= 1024, bf16 inputs).
+// state-major (sm_100a; d_k, d_v in {64, 128, 256}, T_max <= 12, B <= 1024, bf16 inputs).
 //
 // Mathematics ("Scientific Impact Assessment: OneLA", §1 Core Contribution: one shared
 // post-prefill state, append-only transition records, projection replay through the key and
@@ -20,20 +20,27 @@
 // Cf too, so each product runs as hi*hi + lo*hi + hi*lo with fp32 accumulation (the "bf16x2"
 // split of Henry, Tang & Heinecke 2019).
 //
-// One CTA per SM walks the units of its (request, head) pairs, dealt round-robin, through a
-// three-stage operand ring and a four-slot ring of v rows and unit headers. Warp roles:
+// Rows of the state never mix: u_p[i], w_p[i] and o_p[i] use row i of S_ctx and of the w
+// records only, while G and Cf depend on the keys alone. A state of d_v = 256 rows is therefore
+// decoded as two independent blocks of 128 rows (each a (request, head, row block) walk item with
+// its own S_ctx rows in tensor memory; G is formed in both), and d_v = 64 as one block whose
+// M = 128 tensor-core rows 64..127 hold zeros (S_ctx) or are never read (D2).
+//
+// One CTA per SM walks the units of its (request, head, row block) items, dealt round-robin,
+// through an operand ring (three stages, two at d_k = 256) and a ring of v rows and unit
+// headers (four slots, three at d_k = 256). Warp roles:
 //   warps 0-2, 4-5  producers: TMA row gathers (tile::gather4, 128-byte swizzle) of the unit's
 //               q, k and v rows, distinct ancestor keys and w records (the latter as the
 //               MN-major operand), one list of copies dealt out in five chunks; cp.async of
 //               the per-position scalars.
 //   warp 3      head MMA: G with the staged q, k tile as A and the ancestor keys as B; D1 with
 //               S_ctx (bf16 hi + lo) held in tensor memory as the A operand. Three accumulator
-//               stages.
+//               stages (two at d_k = 256, where S_ctx takes 256 tensor-memory columns).
 //   warp 6      tail MMA: D2 with the staged w planes as the A operand and Cf as B, written
 //               over G.
-//   warp 7      prep: decay table, per-position scalars, append of alpha_p.
-//   warps 8-11  coefficients: S_ctx into tensor memory when the (request, head) changes;
-//               k_p . q_p and the append of k_p; Cf from G and the decay table.
+//   warp 7      prep: decay table, per-position scalars, append of alpha_p (row block 0).
+//   warps 8-11  coefficients: S_ctx into tensor memory when the walk item changes;
+//               k_p . q_p and the append of k_p (row block 0); Cf from G and the decay table.
 //   warps 12-19 epilogue: thread = state row i; w_p[i] and o_p[i] from D1, D2 and the scalars;
 //               stores o (fp32) and the w record (hi, lo).
 // Every wait is bounded; on timeout the kernel records OLA_ERR_TIMEOUT and finishes.
@@ -41,12 +48,21 @@
 
 namespace ola {
 
-constexpr int kMmaStages = 3;    // operand stages in shared memory (q / k tile, keys, w planes)
-constexpr int kMmaVSlots = 4;    // v / unit-header slots (held until the epilogue is done)
-constexpr int kMmaAcc = 3;       // accumulator stages in tensor memory (and scalar / decay buffers)
 constexpr int kMmaMaxT = 12;
 constexpr int kMmaMaxB = 1024;
-constexpr int kMmaDV = 128;
+
+// Pipeline depths and row blocking for a geometry. Tensor memory: NA accumulator stages of 128
+// columns, then S_ctx hi | lo (DK columns); shared memory: NS operand stages and NB v slots.
+template <int DK, int DV>
+struct MmaCfg {
+  static constexpr int NRB = DV > 128 ? DV / 128 : 1;   // 128-row blocks of the state
+  static constexpr int DVB = DV < 128 ? DV : 128;       // state rows of one block
+  static constexpr int NVH = DVB / 64;                  // 64-column halves of a block's v row
+  static constexpr int NS = DK > 128 ? 2 : 3;
+  static constexpr int NB = DK > 128 ? 3 : 4;
+  static constexpr int NA = DK > 128 ? 2 : 3;
+  static_assert(128 * NA + DK <= 512, "tensor memory: accumulators and S_ctx");
+};
 // A TMA instruction holds its warp for several hundred cycles plus roughly eighty per active
 // lane, while the instructions of different warps proceed in parallel: the copies of a unit are
 // spread over five producer warps, one warp-wide gather instruction each.
@@ -74,7 +90,7 @@ __device__ __forceinline__ int rec_row_hm(const StepArgs& a, int slot, int r, in
 
 struct MmaInfo {                 // per stage
   int r, h, start, n_pos;
-  int U, first, last, pad;
+  int U, first, last, rb;        // rb: row block of the walk item
   int beam[kUnitPos];
   float gb[2 * kUnitPos];        // (g, beta) of each position
   float alpha[kUnitAnc];         // alpha of each distinct record
@@ -89,49 +105,58 @@ struct MmaScal {                 // per position
 // Shared memory (every tile 1024-byte aligned). The operand stages are released once the
 // unit's MMAs and the coefficient warps are done with them; the v slots and unit headers, read
 // by the epilogue, live in a deeper ring of their own.
-//   operand stage s < 3: X [NSL][64 rows: q of positions 0-31 | k of positions 0-31][128 B]
-//                          K-major, sw128
-//                        KA [NSL][48 rows][128 B]   ancestor keys, same swizzle
-//                        WH, WL [6 groups of 8 records][2 halves of d_v][8][128 B]  MN-major
-//   v slot b < 4: V [2 halves of d_v][32 positions][128 B]  sw128
-//   MmaInfo [4], then CH, CL [64 rows][128 B] (Cf hi, lo; K-major, sw128), DEC [2][32][48]
-//   fp32, SC [3][32], barriers.
+//   operand stage s < NS: X [NSL][64 rows: q of positions 0-31 | k of positions 0-31][128 B]
+//                           K-major, sw128
+//                         KA [NSL][48 rows][128 B]   ancestor keys, same swizzle
+//                         WH, WL [6 groups of 8 records][2 halves of the row block][8][128 B]
+//                           MN-major (at d_v = 64 the second half stays zero)
+//   v slot b < NB: V [NVH halves of the row block][32 positions][128 B]  sw128
+//   MmaInfo [NB], then CH, CL [64 rows][128 B] (Cf hi, lo; K-major, sw128), DEC [2][32][48]
+//   fp32, SC [NA][32], barriers.
 struct MmaLayout {
   uint32_t ka_off, wh_off, wl_off, stage, v_off, info_off;
   uint32_t ch_off, cl_off, dec_off, sc_off, bar_off, bytes;
 };
 
-__host__ __device__ inline MmaLayout mma_layout(int d_k) {
+__host__ __device__ inline MmaLayout mma_layout(int d_k, int nvh, int ns, int nb, int na) {
   const uint32_t NSL = uint32_t(d_k) / 64u;
   MmaLayout L;
   L.ka_off = NSL * 8192u;
   L.wh_off = L.ka_off + NSL * uint32_t(kUnitAnc) * 128u;
   L.wl_off = L.wh_off + uint32_t(kUnitAnc / 8) * 2048u;
   L.stage = L.wl_off + uint32_t(kUnitAnc / 8) * 2048u;
-  L.v_off = uint32_t(kMmaStages) * L.stage;
-  L.info_off = L.v_off + uint32_t(kMmaVSlots) * kUnitPos * kMmaDV * 2u;
-  L.ch_off = (L.info_off + uint32_t(kMmaVSlots) * uint32_t(sizeof(MmaInfo)) + 1023u) & ~1023u;
+  L.v_off = uint32_t(ns) * L.stage;
+  L.info_off = L.v_off + uint32_t(nb * nvh) * kUnitPos * 128u;
+  L.ch_off = (L.info_off + uint32_t(nb) * uint32_t(sizeof(MmaInfo)) + 1023u) & ~1023u;
   L.cl_off = L.ch_off + 8192u;
   L.dec_off = L.cl_off + 8192u;
   L.sc_off = L.dec_off + 2u * kUnitPos * kUnitAnc * 4u;
-  L.bar_off = L.sc_off + uint32_t(kMmaAcc) * kUnitPos * uint32_t(sizeof(MmaScal));
+  L.bar_off = L.sc_off + uint32_t(na) * kUnitPos * uint32_t(sizeof(MmaScal));
   L.bytes = L.bar_off + 320u + 1024u;
   return L;
 }
 
-template <int DK>
+template <int DK, int DV>
+__host__ __device__ inline MmaLayout mma_layout_of() {
+  using C = MmaCfg<DK, DV>;
+  return mma_layout(DK, C::NVH, C::NS, C::NB, C::NA);
+}
+
+template <int DK, int DV>
 __global__ void __launch_bounds__(kMmaWarps * 32, 1)
 replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* __restrict__ S_lo,
                   StepArgs a, UnitPlan up, const __grid_constant__ CUtensorMap mq,
                   const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                   const __grid_constant__ CUtensorMap mkr, const __grid_constant__ CUtensorMap mw) {
-  constexpr int NS = kMmaStages, NB = kMmaVSlots, NA = kMmaAcc, DV = kMmaDV, UC = kUnitAnc,
-                NP = kUnitPos;
+  using Cfg = MmaCfg<DK, DV>;
+  constexpr int NS = Cfg::NS, NB = Cfg::NB, NA = Cfg::NA, UC = kUnitAnc, NP = kUnitPos;
+  constexpr int NRB = Cfg::NRB, DVB = Cfg::DVB, NVH = Cfg::NVH;
+  constexpr int MP = NRB * 128;    // rows of S_hi / S_lo per (request, head)
   constexpr int CR = DK / 8;       // 16-byte chunks of a key row
   constexpr int NSL = DK / 64;     // 64-column slices of a key row
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = align_smem_1024(smem_raw);
-  const MmaLayout L = mma_layout(DK);
+  const MmaLayout L = mma_layout_of<DK, DV>();
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* fullA = bars;              // [NS] operand stage loaded: header arrive + TMA bytes
   uint64_t* emptyA = fullA + NS;       // [NS] operand stage consumed: 2 MMA commits, coef warps
@@ -150,7 +175,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
   uint32_t* holder = reinterpret_cast<uint32_t*>(sfree + 1);
   static_assert((2 * NS + 2 * NB + 4 * NA + 8) * 8 + 8 <= 320, "barrier area");
   auto stage = [&](int s) { return smem + size_t(s) * L.stage; };
-  auto vslot = [&](int b) { return smem + L.v_off + size_t(b) * (NP * DV * 2); };
+  auto vslot = [&](int b) { return smem + L.v_off + size_t(b) * (NP * NVH * 128); };
   auto info = [&](int b) { return reinterpret_cast<MmaInfo*>(smem + L.info_off) + b; };
   unsigned char* CH = smem + L.ch_off;
   unsigned char* CL = smem + L.cl_off;
@@ -159,11 +184,13 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t = a.t, n_anc = t - 1;
-  // (request, head) pairs dealt round-robin: CTA c takes rh = c, c + G, c + 2G, ... so that at
-  // any time the CTAs work on neighbouring heads of the same beams (whose q, k, v, o rows and
-  // records lie next to each other in memory)
+  // walk items (request, head, row block), row block fastest, dealt round-robin: CTA c takes
+  // items c, c + G, c + 2G, ... so that at any time the CTAs work on the row blocks and
+  // neighbouring heads of the same beams (whose q, k, v, o rows and records lie next to each
+  // other in memory, and whose q / k rows a second row block finds in L2)
+  const int n_items = a.R * a.H * NRB;
   int n_my = 0;
-  for (int rh = blockIdx.x; rh < a.R * a.H; rh += gridDim.x) n_my += __ldcg(up.ucnt + rh / a.H);
+  for (int it = blockIdx.x; it < n_items; it += gridDim.x) n_my += __ldcg(up.ucnt + it / (a.H * NRB));
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -206,12 +233,12 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     const int pw = warp < kMmaWMma ? warp : warp - 1;     // 0..4
     int issued = 0;
     if (n_my > 0) {
-      int r = int(blockIdx.x) / a.H, h = int(blockIdx.x) % a.H, k = 0;
-      const int dr = int(gridDim.x) / a.H, dh = int(gridDim.x) % a.H;   // the walk's stride
+      int it = int(blockIdx.x), k = 0;
+      int r = it / (a.H * NRB), h = (it / NRB) % a.H, rb = it % NRB;
       int cnt = __ldcg(up.ucnt + r);
       const int* rec = up.urec + (size_t(r) * up.maxU + k) * kUnitRecInts;
       int x0 = __ldcg(rec + lane), x1 = __ldcg(rec + 32 + lane), x2 = __ldcg(rec + 64 + lane);
-      int prev_rh = -1;
+      int prev_it = -1;
       for (int i = 0; i < n_my; ++i) {
         const int s = i % NS, n = i / NS, sb = i % NB, nb = i / NB;
         bool okw = i < NS || mbar_wait_bounded(&emptyA[s], (n - 1) & 1);
@@ -221,15 +248,13 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           break;
         }
         // the next unit of the walk; its record is fetched now and used in the next iteration
-        int nr = r, nh = h, nk = k + 1, ncnt = cnt;
+        int nit = it, nr = r, nh = h, nrb = rb, nk = k + 1, ncnt = cnt;
         if (nk == cnt) {
           nk = 0;
-          nr = r + dr;
-          nh = h + dh;
-          if (nh >= a.H) {
-            nh -= a.H;
-            ++nr;
-          }
+          nit = it + int(gridDim.x);
+          nr = nit / (a.H * NRB);
+          nh = (nit / NRB) % a.H;
+          nrb = nit % NRB;
         }
         const bool more = i + 1 < n_my;
         int y0 = 0, y1 = 0, y2 = 0;
@@ -240,26 +265,26 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           y1 = __ldcg(nrec + 32 + lane);
           y2 = __ldcg(nrec + 64 + lane);
         }
-        const int rh = r * a.H + h;
-        const int first = rh != prev_rh;
+        const int first = it != prev_it;
         if (first) {
-          // S_ctx hi/lo rows of this (request, head) (first unit only) and of the next one,
-          // into L2 ahead of the builders' loads: 2 x 128 rows x 2 d_k bytes
-          const int npf = (prev_rh < 0 ? 2 : 1);
+          // S_ctx hi/lo rows of this walk item (first unit only) and of the next one, into L2
+          // ahead of the coefficient warps' loads: 2 x DVB rows x 2 d_k bytes
+          const int npf = (prev_it < 0 ? 2 : 1);
           for (int q = 0; q < npf; ++q) {
-            const int rq = rh + (npf == 2 ? q : 1) * int(gridDim.x);
-            if (rq < a.R * a.H) {
-              const unsigned char* hi_b = reinterpret_cast<const unsigned char*>(S_hi) + size_t(rq) * DV * DK * 2;
-              const unsigned char* lo_b = reinterpret_cast<const unsigned char*>(S_lo) + size_t(rq) * DV * DK * 2;
-              for (int x = pw * 32 + lane; x < DV * DK * 2 / 128; x += 32 * kMmaProd) {
+            const int iq = it + (npf == 2 ? q : 1) * int(gridDim.x);
+            if (iq < n_items) {
+              const size_t row0 = size_t(iq / NRB) * MP + size_t(iq % NRB) * 128;
+              const unsigned char* hi_b = reinterpret_cast<const unsigned char*>(S_hi + row0 * DK);
+              const unsigned char* lo_b = reinterpret_cast<const unsigned char*>(S_lo + row0 * DK);
+              for (int x = pw * 32 + lane; x < DVB * DK * 2 / 128; x += 32 * kMmaProd) {
                 prefetch_l2(hi_b + size_t(x) * 128);
                 prefetch_l2(lo_b + size_t(x) * 128);
               }
             }
           }
         }
-        const int last = (!more || nr != r || nh != h) ? 1 : 0;
-        prev_rh = rh;
+        const int last = (!more || nit != it) ? 1 : 0;
+        prev_it = it;
         // record: [0] start | n_pos << 16, [1] U, [4 + p] beam, [36 + u] (slot << 16) | beam
         const int sn = __shfl_sync(kFull, x0, 0);
         const int U = min(__shfl_sync(kFull, x0, 1), UC);
@@ -282,9 +307,12 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         // transaction bytes on fullA[s]; the v rows into the v slot, counted on fullB[sb]. The
         // copies form one list; warp pw issues entries [pw C, pw C + C) in one instruction.
         // Rows past n_pos / U repeat row 0 (never read).
+        // copies: q / k rows (two sides x G4 groups x NSL slices), v rows (G4 groups x NVH
+        // halves), ancestor keys (U4 / 4 groups x NSL slices), w records (U4 / 4 groups x hi, lo
+        // x NVH halves)
         const int U4 = (U + 3) & ~3, G4 = (n_pos + 3) >> 2;
-        const int nqk = 2 * G4 * NSL, nv = 2 * G4, nka = (U4 / 4) * NSL;
-        const int nops = nqk + nv + nka + U4;
+        const int nqk = 2 * G4 * NSL, nv = NVH * G4, nka = (U4 / 4) * NSL;
+        const int nops = nqk + nv + nka + (U4 / 4) * 2 * NVH;
         if (pw == 0) {
           if (lane == 0) {
             inf->r = r;
@@ -294,6 +322,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
             inf->U = U;
             inf->first = first;
             inf->last = last;
+            inf->rb = rb;
           }
           inf->beam[lane] = beam;
           __syncwarp();
@@ -303,10 +332,13 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           }
           __syncwarp();
         }
-        {
-          const int C = (nops + kMmaProd - 1) / kMmaProd;          // <= 24 (<= 120 copies)
-          const int id = pw * C + lane;
-          const bool has = lane < C && id < nops;
+        // warp pw issues entries [pw C, pw C + C), one per lane, 32 at a time (C <= 36: at most
+        // 176 copies at d_k = 256, d_v >= 128)
+        const int C = (nops + kMmaProd - 1) / kMmaProd;
+#pragma unroll 1
+        for (int c0 = 0; c0 < C; c0 += 32) {
+          const int id = pw * C + c0 + lane;
+          const bool has = c0 + lane < C && id < nops;
           const int kind = id < nqk ? 0 : id < nqk + nv ? 1 : id < nqk + nv + nka ? 2 : 3;
           int m, xc;
           unsigned char* dst;
@@ -319,9 +351,9 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
             dst = st + ks * 8192 + (side * NP + 4 * m) * 128;
             map = side ? &mk : &mq;
           } else if (kind == 1) {
-            const int e = id - nqk, ks = e & 1;
-            m = e >> 1;
-            xc = 64 * ks;
+            const int e = id - nqk, ks = e % NVH;
+            m = e / NVH;
+            xc = rb * 128 + 64 * ks;
             dst = vs + ks * (NP * 128) + 4 * m * 128;
             bar = &fullB[sb];
             map = &mv;
@@ -332,9 +364,9 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
             dst = st + L.ka_off + ks * (UC * 128) + 4 * m * 128;
             map = &mkr;
           } else {
-            const int e = id - nqk - nv - nka, pl = (e >> 1) & 1, mb = e & 1;
-            m = e >> 2;
-            xc = 128 * pl + 64 * mb;
+            const int e = id - nqk - nv - nka, mb = e % NVH, pl = (e / NVH) & 1;
+            m = e / (2 * NVH);
+            xc = DV * pl + rb * 128 + 64 * mb;
             dst = st + (pl ? L.wl_off : L.wh_off) + (4 * m >> 3) * 2048 + mb * 1024 + (4 * m & 7) * 128;
             map = &mw;
           }
@@ -363,8 +395,10 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         x0 = y0;
         x1 = y1;
         x2 = y2;
+        it = nit;
         r = nr;
         h = nh;
+        rb = nrb;
         k = nk;
         cnt = ncnt;
       }
@@ -510,7 +544,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         e = x;
         alpha = expf(inf->gb[2 * p]);
         beta = inf->gb[2 * p + 1];
-        a.A[wnew] = alpha;
+        if (inf->rb == 0) a.A[wnew] = alpha;
       }
       sc[p].e = e;
       sc[p].alpha = alpha;
@@ -546,12 +580,12 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         // flight per thread (the rows were prefetched into L2 by the producers)
         tc_fence_after();
         const int row = 32 * sp + lane;
-        const size_t rh = size_t(r) * a.H + h;
+        const size_t srow = (size_t(r) * a.H + h) * MP + size_t(inf->rb) * 128 + row;
         const uint32_t ta = tmem + (uint32_t(32 * sp) << 16) + 128u * NA;
 #pragma unroll 1
         for (int c8 = 0; c8 < DK / 32; ++c8) {          // DK / 64 batches per half
           const int half = c8 / (DK / 64), cb = c8 % (DK / 64);
-          const uint4* src = reinterpret_cast<const uint4*>((half ? S_lo : S_hi) + (rh * DV + row) * DK) + 8 * cb;
+          const uint4* src = reinterpret_cast<const uint4*>((half ? S_lo : S_hi) + srow * DK) + 8 * cb;
           const uint4 w0[4] = {__ldg(src), __ldg(src + 1), __ldg(src + 2), __ldg(src + 3)};
           const uint4 w1[4] = {__ldg(src + 4), __ldg(src + 5), __ldg(src + 6), __ldg(src + 7)};
           tmem_st16(ta + half * (DK / 2) + (2 * cb) * 16, w0);
@@ -589,8 +623,9 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         c0 += __shfl_xor_sync(kFull, c0, 1);
         c0 += __shfl_xor_sync(kFull, c0, 2);
         if (qd == 0) SC[ac * NP + p].c0 = c0;
-        // append k_p: the 128 threads copy the staged k rows (16-byte chunks) into the records
-        const int n_pos = min(inf->n_pos, NP);
+        // append k_p (row block 0 only): the 128 threads copy the staged k rows (16-byte
+        // chunks) into the records
+        const int n_pos = inf->rb == 0 ? min(inf->n_pos, NP) : 0;
 #pragma unroll
         for (int j = 0; j < CR / 4; ++j) {
           const int idx = tc * (CR / 4) + j, pk = idx / CR, c = idx % CR, nn = NP + pk;
@@ -684,7 +719,9 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       const MmaScal* sc = SC + ac * NP;
       const unsigned char* Vb = vslot(sb);          // [2][32][128 B] sw128
       const MmaInfo* inf = info(sb);
-      const int n_pos = min(inf->n_pos, NP), U = inf->U;
+      // rows past the block's DVB (d_v = 64: subpartitions 2, 3) hold nothing to store
+      const int n_pos = row < DVB ? min(inf->n_pos, NP) : 0, U = inf->U;
+      const int orow = inf->rb * 128 + row;           // row of o and of the w record
       const uint32_t base = tl + uint32_t(ac) * 128u;
 #pragma unroll 1
       for (int pb = 0; pb < 2; ++pb) {
@@ -723,11 +760,11 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
                 const float qq = fmaf(sa[jj].x, q1[j], q2[j]);
                 const float w = sa[jj].z * (vv[jj] - sa[jj].y * uu);
                 const float o = fmaf(sa[jj].y, qq, sa[jj].w * w);
-                a.o[size_t(io[jj]) * DV + row] = o;
+                a.o[size_t(io[jj]) * DV + orow] = o;
                 const __nv_bfloat16 whi = __float2bfloat16_rn(w);
                 const __nv_bfloat16 wlo = __float2bfloat16_rn(w - __bfloat162float(whi));
-                Wb[size_t(wn[jj]) * (2 * DV) + row] = whi;
-                Wb[size_t(wn[jj]) * (2 * DV) + DV + row] = wlo;
+                Wb[size_t(wn[jj]) * (2 * DV) + orow] = whi;
+                Wb[size_t(wn[jj]) * (2 * DV) + DV + orow] = wlo;
               }
             }
           }
@@ -751,11 +788,26 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
 
 // ---------------------------------------------------------------------- host side
 
+static bool mma_width(int d) { return d == 64 || d == 128 || d == 256; }
+
 bool replay_mma_supported(int d_k, int d_v, int B, int T_max) {
-  return d_v == kMmaDV && (d_k == 64 || d_k == 128) && T_max <= kMmaMaxT && B <= kMmaMaxB;
+  return mma_width(d_k) && mma_width(d_v) && T_max <= kMmaMaxT && B <= kMmaMaxB;
 }
 
-size_t replay_mma_smem(int d_k) { return mma_layout(d_k).bytes; }
+size_t replay_mma_smem(int d_k, int d_v) {
+  switch (d_k * 1000 + d_v) {
+    case 64064: return mma_layout_of<64, 64>().bytes;
+    case 64128: return mma_layout_of<64, 128>().bytes;
+    case 64256: return mma_layout_of<64, 256>().bytes;
+    case 128064: return mma_layout_of<128, 64>().bytes;
+    case 128128: return mma_layout_of<128, 128>().bytes;
+    case 128256: return mma_layout_of<128, 256>().bytes;
+    case 256064: return mma_layout_of<256, 64>().bytes;
+    case 256128: return mma_layout_of<256, 128>().bytes;
+    case 256256: return mma_layout_of<256, 256>().bytes;
+  }
+  return ~size_t(0);
+}
 
 cudaError_t launch_plan_units(const StepArgs& a, const UnitPlan& up, cudaStream_t stream);
 
@@ -770,14 +822,14 @@ bool make_record_maps(CUtensorMap* mkr, CUtensorMap* mw, const void* Kr, const v
          make_rows_map(mw, W, n_rec, 2 * d_v, uint64_t(d_v) * 4);
 }
 
-template <int DK>
+template <int DK, int DV>
 static cudaError_t launch_mma_t(const void* S_hi, const void* S_lo, const StepArgs& a,
                                 const UnitPlan& up, const CUtensorMap& mq, const CUtensorMap& mk,
                                 const CUtensorMap& mv, const CUtensorMap& mkr, const CUtensorMap& mw,
                                 int n_sm,
                                 cudaStream_t stream) {
-  const MmaLayout L = mma_layout(DK);
-  auto kern = replay_mma_kernel<DK>;
+  const MmaLayout L = mma_layout_of<DK, DV>();
+  auto kern = replay_mma_kernel<DK, DV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(L.bytes));
   if (e != cudaSuccess) return e;
@@ -787,7 +839,8 @@ static cudaError_t launch_mma_t(const void* S_hi, const void* S_lo, const StepAr
   return cudaGetLastError();
 }
 
-// S_hi, S_lo: the shared state split into bf16 hi + lo, [R*H][128][d_k]. W records are stored
+// S_hi, S_lo: the shared state split into bf16 hi + lo, [R*H][M_pad][d_k] (M_pad = d_v rounded
+// up to a multiple of 128, zero rows past d_v). W records are stored
 // as [hi plane | lo plane] bf16 rows of 2 d_v elements. mkr, mw from make_record_maps; the
 // q, k and v maps are made here for this step's inputs.
 cudaError_t launch_replay_mma(const StepArgs& a, const UnitPlan& up, const void* S_hi,
@@ -797,7 +850,7 @@ cudaError_t launch_replay_mma(const StepArgs& a, const UnitPlan& up, const void*
   const uint64_t rows = uint64_t(a.R) * a.B * a.H;
   if (!make_rows_map(&mq, a.q, rows, a.d_k, uint64_t(a.d_k) * 2) ||
       !make_rows_map(&mk, a.k, rows, a.d_k, uint64_t(a.d_k) * 2) ||
-      !make_rows_map(&mv, a.v, rows, kMmaDV, uint64_t(kMmaDV) * 2))
+      !make_rows_map(&mv, a.v, rows, a.d_v, uint64_t(a.d_v) * 2))
     return cudaErrorInvalidValue;
   cudaError_t e = launch_plan_units(a, up, stream);
   if (e != cudaSuccess) return e;
@@ -805,8 +858,21 @@ cudaError_t launch_replay_mma(const StepArgs& a, const UnitPlan& up, const void*
   e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  if (a.d_k == 64) return launch_mma_t<64>(S_hi, S_lo, a, up, mq, mk, mv, mkr, mw, n_sm, stream);
-  if (a.d_k == 128) return launch_mma_t<128>(S_hi, S_lo, a, up, mq, mk, mv, mkr, mw, n_sm, stream);
+#define OLA_MMA_CASE(DK_, DV_)                                                              \
+  case DK_ * 1000 + DV_:                                                                    \
+    return launch_mma_t<DK_, DV_>(S_hi, S_lo, a, up, mq, mk, mv, mkr, mw, n_sm, stream);
+  switch (a.d_k * 1000 + a.d_v) {
+    OLA_MMA_CASE(64, 64)
+    OLA_MMA_CASE(64, 128)
+    OLA_MMA_CASE(64, 256)
+    OLA_MMA_CASE(128, 64)
+    OLA_MMA_CASE(128, 128)
+    OLA_MMA_CASE(128, 256)
+    OLA_MMA_CASE(256, 64)
+    OLA_MMA_CASE(256, 128)
+    OLA_MMA_CASE(256, 256)
+  }
+#undef OLA_MMA_CASE
   return cudaErrorInvalidValue;
 }
 

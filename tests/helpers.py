@@ -18,6 +18,7 @@ PATHS = {
     "replay_fp32": (ola.OLA_PATH_REPLAY, ola.OLA_MATH_FP32),
     "replay_tensor": (ola.OLA_PATH_REPLAY, ola.OLA_MATH_TENSOR),
     "fullstate": (ola.OLA_PATH_FULLSTATE, ola.OLA_MATH_FP32),
+    "replayssm": (ola.OLA_PATH_REPLAYSSM, ola.OLA_MATH_FP32),
 }
 
 

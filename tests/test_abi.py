@@ -63,11 +63,23 @@ def test_workspace_bytes_formula(L):
     g = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, in_dtype=ola.OLA_BF16)
     R, H, dk, dv, B, T = 2, 3, 64, 128, 40, 5
     expect = (R * H * dv * dk * 4 + T * R * H * B * dv * 4 + T * R * H * B * dk * 2 +
-              T * R * H * B * 4 + T * R * B * T * 4 + 16)
+              T * R * H * B * 4 + T * R * B * T * 4 + 16 + R * 4)
     assert ola.ola_workspace_bytes(g) == expect
     gf = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, path=ola.OLA_PATH_FULLSTATE)
     expect_fs = R * H * dv * dk * 4 + 2 * R * H * B * dv * dk * 4 + T * R * B * T * 4 + 16
     assert ola.ola_workspace_bytes(gf) == expect_fs
+    # history-replay path: the raw tokens of every record (k, v in fp32, alpha, beta), no w
+    # records and no per-beam state
+    gr = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, in_dtype=ola.OLA_BF16,
+               path=ola.OLA_PATH_REPLAYSSM)
+    expect_rs = (R * H * dv * dk * 4 + T * R * H * B * dk * 4 + T * R * H * B * 4 +
+                 T * R * H * B * dv * 4 + T * R * H * B * 4 + T * R * B * T * 4 + 16 + R * 4)
+    assert ola.ola_workspace_bytes(gr) == expect_rs
+    # the tensor math is for the record replay path only
+    assert L.ola_workspace_bytes(ctypes.byref(_geom(path=ola.OLA_PATH_REPLAYSSM,
+                                                    in_dtype=ola.OLA_BF16, d_k=128, d_v=128,
+                                                    math=ola.OLA_MATH_TENSOR)),
+                                 ctypes.byref(ctypes.c_uint64(0))) == ola.OLA_ERR_UNSUPPORTED
     # tensor path, d_v = 128: unit plan buffers (counts, prefix, unit records, per-position
     # record indices, a counter) instead of the parent-chain table
     gt = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, in_dtype=ola.OLA_BF16,
@@ -76,14 +88,23 @@ def test_workspace_bytes_formula(L):
     units = R * 4 + (R + 1) * 4 + R * B * 96 * 4 + R * B * 16 + 16
     assert ola.ola_workspace_bytes(gt) == (expect + split + 2 * R * B * 4 + 2 * R * B * 4 +
                                            units)
-    # tensor path, d_v = 64: the parent-chain table
+    # tensor path, d_v = 64: the same unit plan buffers
     dv2 = 64
     g2 = _geom(R=2, H=3, d_k=64, d_v=dv2, B=40, T_max=5, in_dtype=ola.OLA_BF16,
                math=ola.OLA_MATH_TENSOR)
     expect2 = (R * H * dv2 * dk * 4 + T * R * H * B * dv2 * 4 + T * R * H * B * dk * 2 +
-               T * R * H * B * 4 + T * R * B * T * 4 + 16)
+               T * R * H * B * 4 + T * R * B * T * 4 + 16 + R * 4)
     assert ola.ola_workspace_bytes(g2) == (expect2 + 2 * R * H * 128 * dk * 2 + 2 * R * B * 4 +
-                                           2 * R * B * 4 + R * B * T * 4)
+                                           2 * R * B * 4 + units)
+    # tensor path past the unit-planned kernel's chain depth (T_max > 12): the parent-chain
+    # table instead of the unit plan
+    T3 = 13
+    g3 = _geom(R=2, H=3, d_k=64, d_v=dv2, B=40, T_max=T3, in_dtype=ola.OLA_BF16,
+               math=ola.OLA_MATH_TENSOR)
+    expect3 = (R * H * dv2 * dk * 4 + T3 * R * H * B * dv2 * 4 + T3 * R * H * B * dk * 2 +
+               T3 * R * H * B * 4 + T3 * R * B * T3 * 4 + 16 + R * 4)
+    assert ola.ola_workspace_bytes(g3) == (expect3 + 2 * R * H * 128 * dk * 2 + 2 * R * B * 4 +
+                                           2 * R * B * 4 + R * B * T3 * 4)
 
 
 def test_null_arguments(L):

@@ -106,13 +106,13 @@ def test_prefill_zero_tokens_gives_zero_state():
 def test_tiny_all_fp32_paths():
     w = wl.WORKLOADS["tiny"]
     S32, steps, dev_steps, parents = small_problem(w)
-    _check(w, ["replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+    _check(w, ["replay_fp32", "fullstate", "replayssm"], S32, steps, dev_steps, parents)
 
 
 def test_single_request_all_paths():
     w = wl.WORKLOADS["single_request"]
     S32, steps, dev_steps, parents = small_problem(w)
-    _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+    _check(w, ["replay_tensor", "replay_fp32", "fullstate", "replayssm"], S32, steps, dev_steps, parents)
 
 
 @pytest.mark.parametrize("d_k", [64, 128, 256])
@@ -122,35 +122,45 @@ def test_geometries_reduced(d_k, d_v):
     beam count (not a multiple of any chunk) and several tiles."""
     w = wl.WORKLOADS[f"sweep_dk{d_k}_dv{d_v}_B64"].scaled(R=2, H=2, B=100, P=128, T=4)
     S32, steps, dev_steps, parents = small_problem(w)
-    _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+    _check(w, ["replay_tensor", "replay_fp32", "fullstate", "replayssm"], S32, steps, dev_steps, parents)
+
+
+@pytest.mark.parametrize("d_k,d_v", [(64, 64), (128, 64), (256, 128), (64, 256), (256, 256)])
+def test_geometries_past_tensor_unit_limits(d_k, d_v):
+    """T_max = 14 exceeds the chain depth of the unit-planned tensor-core kernel: these handles
+    run the per-chunk tensor-core kernels (d_v = 64: position-major; a 256 in the shape: the
+    d_v-major kernel)."""
+    w = wl.WORKLOADS[f"sweep_dk{d_k}_dv{d_v}_B64"].scaled(R=1, H=2, B=40, P=64, T=14)
+    S32, steps, dev_steps, parents = small_problem(w)
+    _check(w, ["replay_tensor"], S32, steps, dev_steps, parents)
 
 
 @pytest.mark.parametrize("B", [16, 17, 33, 64, 65, 200])
 def test_ragged_beam_counts(B):
     w = wl.WORKLOADS["single_request"].scaled(H=2, B=B, P=64, T=3)
     S32, steps, dev_steps, parents = small_problem(w)
-    _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+    _check(w, ["replay_tensor", "replay_fp32", "fullstate", "replayssm"], S32, steps, dev_steps, parents)
 
 
 @pytest.mark.parametrize("B", [1, 5, 31, 32, 63])
 def test_small_beam_counts_all_paths(B):
     w = wl.WORKLOADS["single_request"].scaled(H=2, B=B, P=32, T=4)
     S32, steps, dev_steps, parents = small_problem(w)
-    _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+    _check(w, ["replay_tensor", "replay_fp32", "fullstate", "replayssm"], S32, steps, dev_steps, parents)
 
 
 @pytest.mark.parametrize("B", [1, 3, 8])
 def test_tiny_beam_counts_fp32(B):
     w = wl.WORKLOADS["tiny"].scaled(B=B, T=4)
     S32, steps, dev_steps, parents = small_problem(w)
-    _check(w, ["replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+    _check(w, ["replay_fp32", "fullstate", "replayssm"], S32, steps, dev_steps, parents)
 
 
 def test_max_steps_32():
     """T_max = 32 (the largest a handle holds): chains as long as a warp."""
     w = wl.WORKLOADS["single_request"].scaled(H=1, B=24, P=16, T=32)
     S32, steps, dev_steps, parents = small_problem(w)
-    _check(w, ["replay_tensor", "replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+    _check(w, ["replay_tensor", "replay_fp32", "fullstate", "replayssm"], S32, steps, dev_steps, parents)
 
 
 @pytest.mark.parametrize("d_k", [64, 128])
@@ -175,7 +185,7 @@ def test_beam_count_limit_of_tensor_units(B):
 def test_bf16_inputs_small_widths_fp32_path():
     w = wl.WORKLOADS["tiny"].scaled(dtype="bf16", d_k=32, d_v=16, B=12)
     S32, steps, dev_steps, parents = small_problem(w)
-    _check(w, ["replay_fp32", "fullstate"], S32, steps, dev_steps, parents)
+    _check(w, ["replay_fp32", "fullstate", "replayssm"], S32, steps, dev_steps, parents)
 
 
 # ----------------------------------------------------------------------------- properties
@@ -337,7 +347,7 @@ def _converging_parents(w, merge_steps):
     return par
 
 
-@pytest.mark.parametrize("path", ["replay_tensor", "replay_fp32"])
+@pytest.mark.parametrize("path", ["replay_tensor", "replay_fp32", "replayssm"])
 def test_compact_decodes_past_t_max(path):
     """A decode of 8 steps on a handle of T_max = 4: ola_compact after steps 3 and 6 folds the
     chain slots every beam shares into S_ctx, and the outputs of every step still match the
@@ -394,3 +404,51 @@ def test_compact_without_shared_prefix_changes_nothing():
     finally:
         dec.close()
     assert max_abs(torch.stack(outs).double().numpy(), ref) <= tol_for("replay_tensor")
+
+
+def _shared_prefix(table):
+    """Chain slots every beam of one request shares: the first slot whose record differs
+    between two beams (table: [B, t] record beam index per slot)."""
+    for s in range(table.shape[1]):
+        if len(np.unique(table[:, s])) > 1:
+            return s
+    return table.shape[1]
+
+
+@pytest.mark.parametrize("path", ["replay_tensor", "replay_fp32", "replayssm"])
+def test_compact_requests_converging_at_different_steps(path):
+    """Three requests whose beams converge at different steps (each request's own merges), a
+    handle of T_max = 4 decoding 9 steps with ola_compact after every step: each call folds the
+    slots every request shares (the smallest shared prefix over the requests, which the oracle's
+    chains give), the decode runs past T_max, and every step matches the oracle."""
+    w = wl.WORKLOADS["single_request"].scaled(R=3, H=2, B=24, P=64, T=9)
+    S32, steps, dev_steps, _ = small_problem(w)
+    parents = wl.make_parents(w)
+    for r, merges in enumerate(([1, 3, 5, 7], [2, 4, 6], [1, 2, 4, 6, 7])):
+        for t in merges:
+            parents[t, r] = 0
+    ref = oracle_outputs(S32, steps, parents)
+    p, m = PATHS[path]
+    dev = torch.device("cuda")
+    dec = ola.Decoder(S32.cuda(), B=w.B, T_max=4, in_dtype=w.torch_dtype, path=p, math=m)
+    outs, base = [], 0                  # base: slots folded so far
+    try:
+        for t in range(w.T):
+            s = dev_steps[t]
+            outs.append(dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"],
+                                 torch.from_numpy(parents[t]).to(dev)).cpu())
+            table = oracle.ancestry_table(parents[: t + 1])[:, :, base:]
+            expect = min(min(_shared_prefix(table[r]) for r in range(w.R)), t - base)
+            got = dec.compact()
+            assert got == expect, (t, got, expect)
+            base += got
+            assert dec.t == t + 1 - base
+        anc = dec.ancestry().cpu().numpy()
+        assert dec.error() == ola.OLA_OK
+    finally:
+        dec.close()
+    assert base >= w.T - 4
+    o = torch.stack(outs).double().numpy()
+    err = max_abs(o, ref)
+    assert err <= tol_for(path), (path, err)
+    assert np.array_equal(anc, oracle.ancestry_table(parents)[:, :, base:])

@@ -52,14 +52,6 @@ def test_step_inputs_distributions():
     assert not torch.equal(x["q"], z["q"])
 
 
-def test_shard_requests_cover():
-    for R in (1, 7, 64):
-        for world in (1, 2, 3, 8):
-            spans = [wl.shard_requests(R, world, r) for r in range(world)]
-            assert spans[0][0] == 0 and spans[-1][1] == R
-            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
-
-
 def test_distinct_ancestor_counts_brute_force():
     W = wl.WORKLOADS["stress"].scaled(R=2, B=32, T=5, max_children=6)
     par = wl.make_parents(W)
