@@ -215,10 +215,17 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = wl.WORKLOADS[args.workload]
     cores = len(os.sched_getaffinity(0))
-    n_units = max(2, 2 * cores)
     pool = _pool(cores)
+    for name in args.workload.split(","):
+        reference_line(wl.WORKLOADS[name], args, pool, cores)
+    pool.close()
+    return 0
+
+
+def reference_line(w: wl.Workload, args, pool, cores) -> None:
+    """The oracle on the host cores, timed on a bounded sample of workload `w`."""
+    n_units = min(w.R * w.H, args.cpu_units or max(2, 2 * cores))
     units = sample_units(w, n_units)
     import torch
     prompt = wl.make_prompt(w.scaled(R=max(r for r, _ in units) + 1), "cpu")
@@ -233,7 +240,6 @@ def run_reference(args):
         dt, n = oracle_sample(w, pu, su, pa, pool, cores)
         times.append(dt)
         work = n
-    pool.close()
     total = sum(times)
     value = work * args.steps / total
     sample = (f"{n_units} of {w.R * w.H} (request, head) units, all {w.B} beams x {w.T} steps; "
@@ -249,7 +255,6 @@ def run_reference(args):
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
-    return 0
 
 
 def describe(w: wl.Workload) -> str:
@@ -310,15 +315,49 @@ def run_ours(args):
     def max_ranks(x: float) -> float:
         return max_over_ranks(x, world, dev)
 
-    base = wl.WORKLOADS[args.workload]
-    if args.requests:
-        base = base.scaled(R=args.requests)
-    w = rank_workload(base, rank)
     cores = len(os.sched_getaffinity(0))
     pool = None
     do_cpu = (not args.no_cpu_baseline) and rank == 0 and world == 1
     if do_cpu:
         pool = _pool(cores)                              # spawn before the first GPU call
+    ctx = dict(torch=torch, ola=ola, world=world, rank=rank, local=local, dev=dev,
+               barrier=barrier, max_ranks=max_ranks, cores=cores, pool=pool, do_cpu=do_cpu)
+    for name in args.workload.split(","):
+        base = wl.WORKLOADS[name]
+        if args.requests:
+            base = base.scaled(R=args.requests)
+        result = bench_workload(rank_workload(base, rank), args, ctx)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    if pool is not None:
+        pool.close()
+        pool.join()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def tensor_path_ok(w: wl.Workload) -> bool:
+    return w.dtype == "bf16" and w.d_k in (64, 128, 256) and w.d_v in (64, 128, 256)
+
+
+def replay_kernel_label(w: wl.Workload) -> str:
+    """The kernels one ola_step launches on the tensor path for this geometry."""
+    if w.d_k in (64, 128, 256) and w.d_v in (64, 128, 256) and w.B <= 1024 and w.T <= 12:
+        return f"ola::plan_units_kernel + ola::replay_mma_kernel<{w.d_k}, {w.d_v}>"
+    if w.d_v == 128 and w.d_k <= 128:
+        return f"ola::plan_units_kernel + ola::replay_pipe_kernel<{w.d_k}>"
+    if w.d_v == 64 and w.d_k <= 128:
+        return f"ola::plan_kernel + ola::replay_pos_kernel<{w.d_k}, {w.d_v}, 64>"
+    return "ola::plan_kernel + ola::replay_tc_kernel"
+
+
+def bench_workload(w: wl.Workload, args, ctx) -> dict:
+    """One bench line: the timed decode of workload `w` and its side measurements."""
+    torch, ola, dev = ctx["torch"], ctx["ola"], ctx["dev"]
+    world, rank, local = ctx["world"], ctx["rank"], ctx["local"]
+    barrier, max_ranks = ctx["barrier"], ctx["max_ranks"]
+    cores, pool, do_cpu = ctx["cores"], ctx["pool"], ctx["do_cpu"]
 
     # ---- inputs resident in HBM; shared state by the library's prefill kernel
     prompt = wl.make_prompt(w, dev)
@@ -326,7 +365,7 @@ def run_ours(args):
     steps = [wl.make_step_inputs(w, t, dev) for t in range(w.T)]
     parents = wl.make_parents(w)
     par_dev = [torch.from_numpy(parents[t]).to(dev) for t in range(w.T)]
-    units = sample_units(w, max(2, 2 * cores)) if do_cpu else []
+    units = sample_units(w, min(w.R * w.H, args.cpu_units or max(2, 2 * cores))) if do_cpu else []
     host = host_units(w, prompt, steps, parents, units) if do_cpu else None
     torch.cuda.synchronize()
 
@@ -343,8 +382,11 @@ def run_ours(args):
             if evs is not None:
                 evs[t][1].record(stream)
 
+    # the tensor-core path takes bf16 inputs and widths 64, 128, 256; other workloads (the tiny
+    # fp32 one) decode on the fp32 replay path
+    tensor = tensor_path_ok(w)
     dec = ola.Decoder(S, B=w.B, T_max=w.T, in_dtype=w.torch_dtype, path=ola.OLA_PATH_REPLAY,
-                      math=ola.OLA_MATH_TENSOR)
+                      math=ola.OLA_MATH_TENSOR if tensor else ola.OLA_MATH_FP32)
     for _ in range(args.warmup):
         decode(dec)
     torch.cuda.synchronize()
@@ -382,12 +424,13 @@ def run_ours(args):
     lit_t = state_and_record_bytes_per_step(w, parents)
     achieved = sum(bytes_t) / (per_launch_ms.sum() / 1e3) / 1e9
     flops = tensor_flops_per_step(w) * w.T
-    tensor_time = flops / (peaks["bf16_tflops"] * 1e12)
+    tensor_time = flops / (peaks["bf16_tflops"] * 1e12) if tensor else 0.0
     hbm_time = sum(bytes_t) / (peaks["hbm_gbs"] * 1e9)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"],
                 "traffic": recorded_traffic(w.name),
-                "kernel": "ola_step = ola::plan_units_kernel + ola::replay_mma_kernel<128>",
+                "kernel": "ola_step = " + (replay_kernel_label(w) if tensor else
+                                           "ola::replay_simt_kernel"),
                 "algorithmic_bytes_per_decode": int(sum(bytes_t)),
                 "frac_state_and_records_only": sum(lit_t) / (per_launch_ms.sum() / 1e3) / 1e9 /
                                                peaks["hbm_gbs"],
@@ -398,16 +441,21 @@ def run_ours(args):
 
     result = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
               "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
-              "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+              "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if tensor else "f32",
               "data": "synthetic",
               "config": {"workload": describe(w), "R": w.R, "H": w.H, "d_k": w.d_k,
                          "d_v": w.d_v, "B": w.B, "T": w.T, "P": w.P,
-                         "path": "replay, tcgen05 tensor cores (bf16 hi/lo S_ctx, fp32 "
-                                 "accumulate and epilogue)",
-                         "l2": "no flush: each decode step streams ~1.4 GB (> 126 MB L2)",
+                         "path": ("replay, tcgen05 tensor cores (bf16 hi/lo S_ctx, fp32 "
+                                  "accumulate and epilogue)" if tensor else
+                                  "replay, fp32 on CUDA cores"),
+                         "l2": ("no flush: each decode step streams %.2f GB (> 126 MB L2)"
+                                % (max(bytes_t) / 1e9) if max(bytes_t) > 126e6 else
+                                "no flush: each decode step streams %.0f MB, inside the 126 MB "
+                                "L2 (a small configuration; its time is launch- and "
+                                "latency-bound)" % (max(bytes_t) / 1e6)),
                          "parallelism": f"replicas x{world} (requests sharded, no collective)"},
               "roofline": roofline, "clocks": clocks,
-              "gpu_launches": 2 * w.T * K}
+              "gpu_launches": (2 if tensor else 1) * w.T * K}
 
     # ---- in-library comparisons on the same inputs (not part of the metric)
     comps = {}
@@ -475,8 +523,6 @@ def run_ours(args):
     if do_cpu:
         pu, su, pa = host
         dt, n = oracle_sample(w, pu, su, pa, pool, cores)
-        pool.close()
-        pool.join()
         result["cpu_baseline"] = {
             "value": n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{len(pu)} of {w.R * w.H} (request, head) units of this workload, all "
@@ -493,12 +539,9 @@ def run_ours(args):
         "ms": pf_ms, "algorithmic_bytes": pf_bytes,
         "achieved_gbs": pf_bytes / (pf_ms / 1e3) / 1e9,
         "hbm_frac": pf_bytes / (pf_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
-
-    if rank == 0:
-        print(json.dumps(result), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
-    return 0
+    del S, steps, par_dev, outs, prompt
+    torch.cuda.empty_cache()
+    return result
 
 
 # ----------------------------------------------------------------------------- operator sweep
@@ -651,7 +694,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="stress", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--workload", default="stress",
+                    help="workload name, or several separated by commas (one JSON line each): "
+                         + ", ".join(sorted(wl.WORKLOADS)))
+    ap.add_argument("--cpu-units", type=int, default=0,
+                    help="(request, head) units of the CPU oracle sample (default 2 x cores)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-compare", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -671,6 +718,9 @@ def main():
                     help="also report the largest |o| difference between replay and FullState")
     ap.add_argument("--sweep-no-fullstate", action="store_true")
     args = ap.parse_args()
+    for name in args.workload.split(","):
+        if name not in wl.WORKLOADS:
+            ap.error(f"unknown workload {name}")
     if args.sweep:
         return run_sweep(args)
     if args.warmup < 3 and args.impl == "ours":

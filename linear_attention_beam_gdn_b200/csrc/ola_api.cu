@@ -37,6 +37,7 @@ cudaError_t launch_replay_pipe(const StepArgs& a, const void* S_hi, const void* 
                                cudaStream_t stream);
 bool replay_mma_supported(int d_k, int d_v, int B, int T_max);
 size_t replay_mma_smem(int d_k, int d_v);
+int replay_mma_unit_records(int d_k, int d_v);
 size_t plan_units_smem(int B, int T_max);
 cudaError_t launch_replay_mma(const StepArgs& a, const UnitPlan& up, const void* S_hi,
                               const void* S_lo, const CUtensorMap& mkr, const CUtensorMap& mw,
@@ -160,9 +161,9 @@ Sizes sizes_of(const ola_geometry* g) {
   z.S_split = g->math == OLA_MATH_TENSOR ? R * H * ((dv + 127) / 128 * 128) * dk * 2 : 0;
   const bool rep = g->path == OLA_PATH_REPLAY, rss = g->path == OLA_PATH_REPLAYSSM;
   z.W = rep ? T * R * H * B * dv * 4 : 0;
-  z.Kr = rep ? T * R * H * B * dk * e : rss ? T * R * H * B * dk * 4 : 0;
+  z.Kr = (rep || rss) ? T * R * H * B * dk * e : 0;
   z.A = (rep || rss) ? T * R * H * B * 4 : 0;
-  z.Vr = rss ? T * R * H * B * dv * 4 : 0;
+  z.Vr = rss ? T * R * H * B * dv * e : 0;
   z.Br = rss ? T * R * H * B * 4 : 0;
   z.C = T * R * B * T * 4;
   z.FS = g->path == OLA_PATH_FULLSTATE ? R * H * B * dv * dk * 4 : 0;
@@ -344,6 +345,7 @@ ola_status ola_create(const ola_geometry* geom, const float* S_ctx, void* stream
   if (e == cudaSuccess) e = dev_alloc(&h->up.counter, z.counter);
   if (e == cudaSuccess && z.counter) e = cudaMemsetAsync(h->up.counter, 0, z.counter, st);
   h->up.maxU = geom->B;
+  h->up.maxAnc = replay_mma_unit_records(geom->d_k, geom->d_v);
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->S, S_ctx, z.S, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, z.err, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->C, 0, z.C, st);
@@ -528,15 +530,15 @@ ola_status ola_compact(ola_handle h, int32_t* out_folded, void* stream) {
   // and the chain rows down by c
   const bool rss = g.path == OLA_PATH_REPLAYSSM;
   const int layout = rss ? 2 : h->mma ? 1 : 0;
-  e = launch_fold(h->S, rss ? h->Vr : h->W, h->Kr, !rss && g.in_dtype == OLA_BF16, h->A, h->Br,
-                  h->C, g.R, g.H, g.d_k, g.d_v, g.B, g.T_max, t, c, layout, st);
+  e = launch_fold(h->S, rss ? h->Vr : h->W, h->Kr, g.in_dtype == OLA_BF16, h->A, h->Br, h->C,
+                  g.R, g.H, g.d_k, g.d_v, g.B, g.T_max, t, c, layout, st);
   if (e == cudaSuccess && g.math == OLA_MATH_TENSOR)
     e = launch_split_state(h->S, h->S_hi, h->S_lo, g.R * g.H, g.d_k, g.d_v, st);
   const size_t rows = size_t(g.R) * g.H * g.B;
   const size_t kbytes = g.in_dtype == OLA_BF16 ? 2 : 4;
   // per record slot: w (or, on the history-replay path, v and beta), k, alpha
-  const size_t w_slot = rows * g.d_v * 4;
-  const size_t k_slot = rows * g.d_k * (rss ? 4 : kbytes), a_slot = rows * 4;
+  const size_t w_slot = rss ? rows * g.d_v * kbytes : rows * g.d_v * 4;
+  const size_t k_slot = rows * g.d_k * kbytes, a_slot = rows * 4;
   char* const bufs[4] = {reinterpret_cast<char*>(rss ? h->Vr : h->W), static_cast<char*>(h->Kr),
                          reinterpret_cast<char*>(h->A), reinterpret_cast<char*>(h->Br)};
   const size_t slot_bytes[4] = {w_slot, k_slot, a_slot, rss ? a_slot : 0};

@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(256) common_prefix_kernel(const int* __restric
 //   layout 0: records [T_max][R][H][B], w fp32 [d_v]
 //   layout 1: records [T_max][R][B][H], w as bf16 hi and lo planes [2][d_v]
 //   layout 2: records [T_max][R][H][B] holding the raw token (history-replay path): k and v
-//             in fp32, and beta; w_j[i] = beta_j (v_j[i] - alpha_j S_i . k_j) is formed
+//             in the input dtype, and beta; w_j[i] = beta_j (v_j[i] - alpha_j S_i . k_j) is formed
 //             from the state folded so far (the gated delta rule itself)
 template <typename TK>
 __global__ void __launch_bounds__(128) fold_kernel(float* __restrict__ S, const void* __restrict__ Wp,

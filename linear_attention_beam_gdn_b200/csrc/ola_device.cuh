@@ -43,14 +43,14 @@ struct StepArgs {
   const int* rank_prev;         // [R][B] depth-first position of each beam of step t-1
   int* rank_cur;                // [R][B] depth-first position of each beam of step t
   int* err;                     // device error word: [0] code, [1] detail, [2] step
-  // history-replay path only: the raw tokens of every step (Kr holds the keys, in fp32)
-  void* Vr;                     // [T_max][R][H][B][d_v] fp32      v_t
+  // history-replay path only: the raw tokens of every step (Kr holds the keys)
+  void* Vr;                     // [T_max][R][H][B][d_v] in_dtype  copy of v_t
   float* Br;                    // [T_max][R][H][B]      fp32      beta_t
 };
 
 // Units of work of the tensor-core replay kernel, written each step by plan_units_kernel
 // (ola_plan.cu): at most kUnitPos consecutive depth-first positions of one request whose
-// parent chains reach at most kUnitAnc distinct records.
+// parent chains reach at most maxAnc <= kUnitAnc distinct records.
 constexpr int kUnitPos = 32;
 constexpr int kUnitAnc = 48;
 constexpr int kUnitRecInts = 96;
@@ -62,6 +62,7 @@ struct UnitPlan {
   uint8_t* upos;      // [R][B][16]
   unsigned* counter;  // CTAs finished (reset to 0 by the last one)
   int maxU;           // units per request at most
+  int maxAnc;         // distinct records per unit at most (<= kUnitAnc; the replay kernel's)
 };
 
 

@@ -73,7 +73,7 @@ cudaError_t launch_plan(const StepArgs& a, cudaStream_t stream) {
 // Depth-first positions cut into units for the tensor-core replay kernel (ola_replay_mma.cu).
 //
 // A unit is a run of at most kUnitPos consecutive depth-first positions of one request whose
-// parent chains reach at most kUnitAnc distinct records. In depth-first order every record's
+// parent chains reach at most up.maxAnc distinct records. In depth-first order every record's
 // descendants are contiguous, so within a chain slot the records of consecutive positions are
 // equal or new, and the distinct records of a unit are the slot-wise changes. Units are made of
 // whole sibling groups where they fit (see the cut below).
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up
   __syncthreads();
   // units. Beams with the same parent have the same chain, and their outputs must not depend on
   // how the beams are cut into units: a unit holds whole sibling groups of at most kUnitPos
-  // positions while its distinct records stay <= kUnitAnc (greedy, left to right); a larger
+  // positions while its distinct records stay <= up.maxAnc (greedy, left to right); a larger
   // group is cut into chunks of kUnitPos positions, each a unit of its own, so that every chunk
   // lists the chain's records in the same order (record u = chain slot u). A unit starting at
   // group g takes n_anc records for its first group and popc(fnew) new ones for each further
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up
       int lo = g + 1, hi = ng;
       while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        const bool viol = PS[mid + 1] - PS[g] > kUnitPos || n_anc + PC[mid + 1] - PC[g + 1] > kUnitAnc;
+        const bool viol = PS[mid + 1] - PS[g] > kUnitPos || n_anc + PC[mid + 1] - PC[g + 1] > up.maxAnc;
         if (viol) hi = mid;
         else lo = mid + 1;
       }

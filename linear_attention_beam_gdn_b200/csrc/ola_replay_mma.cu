@@ -23,8 +23,11 @@
 // Rows of the state never mix: u_p[i], w_p[i] and o_p[i] use row i of S_ctx and of the w
 // records only, while G and Cf depend on the keys alone. A state of d_v = 256 rows is therefore
 // decoded as two independent blocks of 128 rows (each a (request, head, row block) walk item with
-// its own S_ctx rows in tensor memory; G is formed in both), and d_v = 64 as one block whose
-// M = 128 tensor-core rows 64..127 hold zeros (S_ctx) or are never read (D2).
+// its own S_ctx rows in tensor memory; G is formed in both). At d_v = 64 the M = 128 tensor-core
+// rows hold the state twice (S_ctx rows 0..63 again in tensor-memory lanes 64..127, and the w
+// planes' second 64-row block read from the first one): D1 and D2 then carry every position in
+// both halves, and the epilogue warps of lanes 0..63 finish positions 0..15 while those of lanes
+// 64..127 finish positions 16..31, so all eight epilogue warps share the unit.
 //
 // One CTA per SM walks the units of its (request, head, row block) items, dealt round-robin,
 // through an operand ring (three stages, two at d_k = 256) and a ring of v rows and unit
@@ -51,17 +54,21 @@ namespace ola {
 constexpr int kMmaMaxT = 12;
 constexpr int kMmaMaxB = 1024;
 
-// Pipeline depths and row blocking for a geometry. Tensor memory: NA accumulator stages of 128
-// columns, then S_ctx hi | lo (DK columns); shared memory: NS operand stages and NB v slots.
+// Pipeline depths, unit size and row blocking for a geometry. Tensor memory: NA accumulator
+// stages of 128 columns, then S_ctx hi | lo (DK columns); shared memory: NS operand stages of
+// which the ancestor keys and w planes are sized for UC records, and NB v slots. A unit holds at
+// most UC distinct ancestor records (the plan cuts units to that).
 template <int DK, int DV>
 struct MmaCfg {
   static constexpr int NRB = DV > 128 ? DV / 128 : 1;   // 128-row blocks of the state
   static constexpr int DVB = DV < 128 ? DV : 128;       // state rows of one block
   static constexpr int NVH = DVB / 64;                  // 64-column halves of a block's v row
+  static constexpr int UC = kUnitAnc;
   static constexpr int NS = DK > 128 ? 2 : 3;
   static constexpr int NB = DK > 128 ? 3 : 4;
   static constexpr int NA = DK > 128 ? 2 : 3;
   static_assert(128 * NA + DK <= 512, "tensor memory: accumulators and S_ctx");
+  static_assert(UC % 16 == 0 && UC <= kUnitAnc, "records come in MMA K-steps of 16");
 };
 // A TMA instruction holds its warp for several hundred cycles plus roughly eighty per active
 // lane, while the instructions of different warps proceed in parallel: the copies of a unit are
@@ -118,19 +125,20 @@ struct MmaLayout {
   uint32_t ch_off, cl_off, dec_off, sc_off, bar_off, bytes;
 };
 
-__host__ __device__ inline MmaLayout mma_layout(int d_k, int nvh, int ns, int nb, int na) {
+__host__ __device__ inline MmaLayout mma_layout(int d_k, int nvh, int ns, int nb, int na,
+                                                int uc) {
   const uint32_t NSL = uint32_t(d_k) / 64u;
   MmaLayout L;
   L.ka_off = NSL * 8192u;
-  L.wh_off = L.ka_off + NSL * uint32_t(kUnitAnc) * 128u;
-  L.wl_off = L.wh_off + uint32_t(kUnitAnc / 8) * 2048u;
-  L.stage = L.wl_off + uint32_t(kUnitAnc / 8) * 2048u;
+  L.wh_off = L.ka_off + NSL * uint32_t(uc) * 128u;
+  L.wl_off = L.wh_off + uint32_t(uc / 8) * 2048u;
+  L.stage = L.wl_off + uint32_t(uc / 8) * 2048u;
   L.v_off = uint32_t(ns) * L.stage;
   L.info_off = L.v_off + uint32_t(nb * nvh) * kUnitPos * 128u;
   L.ch_off = (L.info_off + uint32_t(nb) * uint32_t(sizeof(MmaInfo)) + 1023u) & ~1023u;
   L.cl_off = L.ch_off + 8192u;
   L.dec_off = L.cl_off + 8192u;
-  L.sc_off = L.dec_off + 2u * kUnitPos * kUnitAnc * 4u;
+  L.sc_off = L.dec_off + 2u * kUnitPos * uint32_t(uc) * 4u;
   L.bar_off = L.sc_off + uint32_t(na) * kUnitPos * uint32_t(sizeof(MmaScal));
   L.bytes = L.bar_off + 320u + 1024u;
   return L;
@@ -139,7 +147,7 @@ __host__ __device__ inline MmaLayout mma_layout(int d_k, int nvh, int ns, int nb
 template <int DK, int DV>
 __host__ __device__ inline MmaLayout mma_layout_of() {
   using C = MmaCfg<DK, DV>;
-  return mma_layout(DK, C::NVH, C::NS, C::NB, C::NA);
+  return mma_layout(DK, C::NVH, C::NS, C::NB, C::NA, C::UC);
 }
 
 template <int DK, int DV>
@@ -149,7 +157,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
                   const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                   const __grid_constant__ CUtensorMap mkr, const __grid_constant__ CUtensorMap mw) {
   using Cfg = MmaCfg<DK, DV>;
-  constexpr int NS = Cfg::NS, NB = Cfg::NB, NA = Cfg::NA, UC = kUnitAnc, NP = kUnitPos;
+  constexpr int NS = Cfg::NS, NB = Cfg::NB, NA = Cfg::NA, UC = Cfg::UC, NP = kUnitPos;
   constexpr int NRB = Cfg::NRB, DVB = Cfg::DVB, NVH = Cfg::NVH;
   constexpr int MP = NRB * 128;    // rows of S_hi / S_lo per (request, head)
   constexpr int CR = DK / 8;       // 16-byte chunks of a key row
@@ -479,8 +487,10 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         const uint32_t id2 = idesc_bf16_f32_amn(128, 2 * NP);
 #pragma unroll 1
         for (int kq = 0; kq < (U + 15) / 16; ++kq) {
-          const uint64_t ah = sw128_mnmajor_desc(st + L.wh_off + kq * 4096, 1024, 2048);
-          const uint64_t al = sw128_mnmajor_desc(st + L.wl_off + kq * 4096, 1024, 2048);
+          // the two 64-row blocks of the A operand: 1024 bytes apart, or (d_v = 64) the same
+          // block twice
+          const uint64_t ah = sw128_mnmajor_desc(st + L.wh_off + kq * 4096, DVB == 64 ? 0 : 1024, 2048);
+          const uint64_t al = sw128_mnmajor_desc(st + L.wl_off + kq * 4096, DVB == 64 ? 0 : 1024, 2048);
           const uint64_t bh = sw128_kmajor_desc(smem_u32(CH) + kq * 32);
           const uint64_t bl = sw128_kmajor_desc(smem_u32(CL) + kq * 32);
           umma_bf16_w(d2, ah, bh, id2, kq != 0 ? 1u : 0u);
@@ -580,7 +590,8 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         // flight per thread (the rows were prefetched into L2 by the producers)
         tc_fence_after();
         const int row = 32 * sp + lane;
-        const size_t srow = (size_t(r) * a.H + h) * MP + size_t(inf->rb) * 128 + row;
+        // d_v = 64: lanes 64..127 hold S_ctx rows 0..63 again
+        const size_t srow = (size_t(r) * a.H + h) * MP + size_t(inf->rb) * 128 + (row % DVB);
         const uint32_t ta = tmem + (uint32_t(32 * sp) << 16) + 128u * NA;
 #pragma unroll 1
         for (int c8 = 0; c8 < DK / 32; ++c8) {          // DK / 64 batches per half
@@ -705,6 +716,11 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     // thread = state row (tensor-memory lane); warp (sp, ph) = rows 32 sp.., positions 16 ph..
     const int ew = warp - kMmaWEpi, sp = warp & 3, ph = ew >> 2;
     const int row = 32 * sp + lane;
+    // state row this lane finishes, and its positions: [16 ph, 16 ph + 16), or at d_v = 64
+    // (lanes 64..127 repeat rows 0..63) [16 (sp / 2) + 8 ph, + 8)
+    const int drow = row % DVB;
+    const int pbase = DVB == 64 ? 16 * (sp >> 1) + 8 * ph : 16 * ph;
+    constexpr int NPB = DVB == 64 ? 1 : 2;          // batches of 8 positions per warp
     const uint32_t tl = tmem + (uint32_t(32 * sp) << 16);
     __nv_bfloat16* Wb = reinterpret_cast<__nv_bfloat16*>(a.W);
     for (int i = 0; i < n_my; ++i) {
@@ -719,13 +735,12 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       const MmaScal* sc = SC + ac * NP;
       const unsigned char* Vb = vslot(sb);          // [2][32][128 B] sw128
       const MmaInfo* inf = info(sb);
-      // rows past the block's DVB (d_v = 64: subpartitions 2, 3) hold nothing to store
-      const int n_pos = row < DVB ? min(inf->n_pos, NP) : 0, U = inf->U;
-      const int orow = inf->rb * 128 + row;           // row of o and of the w record
+      const int n_pos = min(inf->n_pos, NP), U = inf->U;
+      const int orow = inf->rb * 128 + drow;          // row of o and of the w record
       const uint32_t base = tl + uint32_t(ac) * 128u;
 #pragma unroll 1
-      for (int pb = 0; pb < 2; ++pb) {
-        const int p0 = 16 * ph + 8 * pb;
+      for (int pb = 0; pb < NPB; ++pb) {
+        const int p0 = pbase + 8 * pb;
         if (p0 < n_pos) {                             // warp-uniform
           float q1[8], k1[8], q2[8], k2[8];
           tmem_ld8x4(base + p0, base + NP + p0, base + 2 * NP + p0, base + 3 * NP + p0, q1, k1,
@@ -749,8 +764,8 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
               io[jj] = sb.x;
               wn[jj] = sb.y;
               vv[jj] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                  Vb + (row >> 6) * (NP * 128) + pp * 128 + ((((row & 63) >> 3) ^ (pp & 7)) << 4) +
-                  (row & 7) * 2));
+                  Vb + (drow >> 6) * (NP * 128) + pp * 128 + ((((drow & 63) >> 3) ^ (pp & 7)) << 4) +
+                  (drow & 7) * 2));
             }
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
@@ -792,6 +807,21 @@ static bool mma_width(int d) { return d == 64 || d == 128 || d == 256; }
 
 bool replay_mma_supported(int d_k, int d_v, int B, int T_max) {
   return mma_width(d_k) && mma_width(d_v) && T_max <= kMmaMaxT && B <= kMmaMaxB;
+}
+
+int replay_mma_unit_records(int d_k, int d_v) {
+  switch (d_k * 1000 + d_v) {
+    case 64064: return MmaCfg<64, 64>::UC;
+    case 64128: return MmaCfg<64, 128>::UC;
+    case 64256: return MmaCfg<64, 256>::UC;
+    case 128064: return MmaCfg<128, 64>::UC;
+    case 128128: return MmaCfg<128, 128>::UC;
+    case 128256: return MmaCfg<128, 256>::UC;
+    case 256064: return MmaCfg<256, 64>::UC;
+    case 256128: return MmaCfg<256, 128>::UC;
+    case 256256: return MmaCfg<256, 256>::UC;
+  }
+  return kUnitAnc;
 }
 
 size_t replay_mma_smem(int d_k, int d_v) {

@@ -20,7 +20,9 @@
 // S^ (S = sigma S^): a transition is then sigma <- alpha sigma, S^ += (w / sigma) k, one fused
 // multiply-add per element instead of a multiply and a fused multiply-add (S^ is rescaled into
 // S whenever sigma falls below 2^-60, so it stays far from fp32 overflow). The keys and values of
-// the history are kept in fp32 (converted once, when they are appended).
+// the history are kept in the input dtype: the rebuilds stream the keys through L1/L2 for every
+// beam, so their bytes, not the conversion, set the pace (measured: fp32 keys made the stress
+// decode 1.3x slower).
 //
 // Grid: (request, head) x blocks of state rows. A CTA of 8 warps holds its rows of S_ctx in
 // shared memory (read from HBM once per step and CTA) and walks every beam of the request;
@@ -140,10 +142,10 @@ replayssm_kernel(StepArgs a) {
       const size_t in = (size_t(r) * a.B + b) * a.H + h;
       const size_t rec = rec_index(a, slot, r, h, b);
       for (int e = lane; e < DK; e += 32)
-        static_cast<float*>(a.Kr)[rec * DK + e] = to_f32(static_cast<const TIn*>(a.k)[in * DK + e]);
+        static_cast<TIn*>(a.Kr)[rec * DK + e] = static_cast<const TIn*>(a.k)[in * DK + e];
       for (int e = lane; e < a.d_v; e += 32)
-        static_cast<float*>(a.Vr)[rec * a.d_v + e] =
-            to_f32(static_cast<const TIn*>(a.v)[in * size_t(a.d_v) + e]);
+        static_cast<TIn*>(a.Vr)[rec * a.d_v + e] =
+            static_cast<const TIn*>(a.v)[in * size_t(a.d_v) + e];
       if (lane == 0) {
         a.A[rec] = expf(a.g[in]);
         a.Br[rec] = a.beta[in];
@@ -185,8 +187,8 @@ replayssm_kernel(StepArgs a) {
       const int c = __shfl_sync(0xffffffffu, cidx, j < n_anc ? j : 0);
       if (j < n_anc) {
         const size_t rec = rec_index(a, j, r, h, c);
-        load_slice<float, EL>(kx, a.Kr, rec, e0, DK);
-        vx = row_ok ? static_cast<const float*>(a.Vr)[rec * a.d_v + row] : 0.f;
+        load_slice<TIn, EL>(kx, a.Kr, rec, e0, DK);
+        vx = row_ok ? to_f32(static_cast<const TIn*>(a.Vr)[rec * a.d_v + row]) : 0.f;
         ax = __ldg(a.A + rec);
         bx = __ldg(a.Br + rec);
       } else {

@@ -68,12 +68,12 @@ def test_workspace_bytes_formula(L):
     gf = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, path=ola.OLA_PATH_FULLSTATE)
     expect_fs = R * H * dv * dk * 4 + 2 * R * H * B * dv * dk * 4 + T * R * B * T * 4 + 16
     assert ola.ola_workspace_bytes(gf) == expect_fs
-    # history-replay path: the raw tokens of every record (k, v in fp32, alpha, beta), no w
-    # records and no per-beam state
+    # history-replay path: the raw tokens of every record (k, v in the input dtype, alpha,
+    # beta), no w records and no per-beam state
     gr = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, in_dtype=ola.OLA_BF16,
                path=ola.OLA_PATH_REPLAYSSM)
-    expect_rs = (R * H * dv * dk * 4 + T * R * H * B * dk * 4 + T * R * H * B * 4 +
-                 T * R * H * B * dv * 4 + T * R * H * B * 4 + T * R * B * T * 4 + 16 + R * 4)
+    expect_rs = (R * H * dv * dk * 4 + T * R * H * B * dk * 2 + T * R * H * B * 4 +
+                 T * R * H * B * dv * 2 + T * R * H * B * 4 + T * R * B * T * 4 + 16 + R * 4)
     assert ola.ola_workspace_bytes(gr) == expect_rs
     # the tensor math is for the record replay path only
     assert L.ola_workspace_bytes(ctypes.byref(_geom(path=ola.OLA_PATH_REPLAYSSM,
