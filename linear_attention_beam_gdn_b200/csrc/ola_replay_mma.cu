@@ -119,7 +119,7 @@ struct MmaScal {                 // per position
 //                           MN-major (at d_v = 64 the second half stays zero)
 //   v slot b < NB: V [NVH halves of the row block][32 positions][128 B]  sw128
 //   MmaInfo [NB], then CH, CL [64 rows][128 B] (Cf hi, lo; K-major, sw128), DEC [2][32][48]
-//   fp32, SC [NA][32], barriers.
+//   fp32, SC [NB][32] (per-position scalars, by v slot), barriers.
 struct MmaLayout {
   uint32_t ka_off, wh_off, wl_off, stage, v_off, info_off;
   uint32_t ch_off, cl_off, dec_off, sc_off, bar_off, bytes;
@@ -139,7 +139,7 @@ __host__ __device__ inline MmaLayout mma_layout(int d_k, int nvh, int ns, int nb
   L.cl_off = L.ch_off + 8192u;
   L.dec_off = L.cl_off + 8192u;
   L.sc_off = L.dec_off + 2u * kUnitPos * uint32_t(uc) * 4u;
-  L.bar_off = L.sc_off + uint32_t(na) * kUnitPos * uint32_t(sizeof(MmaScal));
+  L.bar_off = L.sc_off + uint32_t(nb) * kUnitPos * uint32_t(sizeof(MmaScal));
   L.bytes = L.bar_off + 320u + 1024u;
   return L;
 }
@@ -172,8 +172,8 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
   uint64_t* emptyB = fullB + NB;       // [NB] v slot consumed: epilogue warps
   uint64_t* acc_full = emptyB + NB;    // [NA] accumulators of a unit complete (D1 and D2 commits)
   uint64_t* acc_empty = acc_full + NA; // [NA] epilogue done with an accumulator stage
-  uint64_t* scal_ready = acc_empty + NA;  // [NA] per-position scalars written
-  uint64_t* g_ready = scal_ready + NA;    // [NA] G of a unit in tensor memory (every unit)
+  uint64_t* scal_ready = acc_empty + NA;  // [NB] per-position scalars written (by v slot)
+  uint64_t* g_ready = scal_ready + NB;    // [NA] G of a unit in tensor memory (every unit)
   uint64_t* dec_ready = g_ready + NA;     // [2] decay table buffer written
   uint64_t* dec_free = dec_ready + 2;     // [2] coefficient warps done with a decay table buffer
   uint64_t* coef_ready = dec_free + 2;    // Cf of the current unit written (every unit)
@@ -181,7 +181,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
   uint64_t* sready = coef_free + 1;    // S_ctx loaded into tensor memory
   uint64_t* sfree = sready + 1;        // last MMA reading S_ctx done
   uint32_t* holder = reinterpret_cast<uint32_t*>(sfree + 1);
-  static_assert((2 * NS + 2 * NB + 4 * NA + 8) * 8 + 8 <= 320, "barrier area");
+  static_assert((2 * NS + 3 * NB + 3 * NA + 8) * 8 + 8 <= 320, "barrier area");
   auto stage = [&](int s) { return smem + size_t(s) * L.stage; };
   auto vslot = [&](int b) { return smem + L.v_off + size_t(b) * (NP * NVH * 128); };
   auto info = [&](int b) { return reinterpret_cast<MmaInfo*>(smem + L.info_off) + b; };
@@ -196,9 +196,10 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
   // items c, c + G, c + 2G, ... so that at any time the CTAs work on the row blocks and
   // neighbouring heads of the same beams (whose q, k, v, o rows and records lie next to each
   // other in memory, and whose q / k rows a second row block finds in L2)
-  const int n_items = a.R * a.H * NRB;
+  const int HN = a.H * NRB;
+  const int n_items = a.R * HN;
   int n_my = 0;
-  for (int it = blockIdx.x; it < n_items; it += gridDim.x) n_my += __ldcg(up.ucnt + it / (a.H * NRB));
+  for (int it = blockIdx.x; it < n_items; it += gridDim.x) n_my += __ldcg(up.ucnt + it / HN);
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -208,12 +209,12 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     for (int b = 0; b < NB; ++b) {
       mbar_init(&fullB[b], 32 * kMmaProd + 1);  // cp.async arrivals + header (with bytes)
       mbar_init(&emptyB[b], kMmaEpi);
+      mbar_init(&scal_ready[b], 1 + kMmaCoef);   // prep warp, c0 from the coefficient warps
     }
     for (int x = 0; x < NA; ++x) {
       mbar_init(&acc_full[x], 2);
       mbar_init(&g_ready[x], 1);
       mbar_init(&acc_empty[x], kMmaEpi);
-      mbar_init(&scal_ready[x], 1 + kMmaCoef);   // prep warp, c0 from the coefficient warps
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&dec_ready[x], 1);
@@ -242,7 +243,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     int issued = 0;
     if (n_my > 0) {
       int it = int(blockIdx.x), k = 0;
-      int r = it / (a.H * NRB), h = (it / NRB) % a.H, rb = it % NRB;
+      int r = it / HN, h = (it / NRB) % a.H, rb = it % NRB;
       int cnt = __ldcg(up.ucnt + r);
       const int* rec = up.urec + (size_t(r) * up.maxU + k) * kUnitRecInts;
       int x0 = __ldcg(rec + lane), x1 = __ldcg(rec + 32 + lane), x2 = __ldcg(rec + 64 + lane);
@@ -260,7 +261,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         if (nk == cnt) {
           nk = 0;
           nit = it + int(gridDim.x);
-          nr = nit / (a.H * NRB);
+          nr = nit / HN;
           nh = (nit / NRB) % a.H;
           nrb = nit % NRB;
         }
@@ -512,7 +513,6 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     for (int i = 0; i < n_my; ++i) {
       const int sb = i % NB, ac = i % NA, db = i & 1;
       bool ok = mbar_wait_bounded(&fullB[sb], (i / NB) & 1);
-      if (i >= NA) ok = ok && mbar_wait_bounded(&acc_empty[ac], ((i - NA) / NA) & 1);  // SC[ac] free
       if (i >= 2) ok = ok && mbar_wait_bounded(&dec_free[db], ((i - 2) >> 1) & 1);      // DEC[db] free
       if (!__all_sync(kFull, ok)) {
         if (lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 23, t);
@@ -520,7 +520,9 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       }
       const MmaInfo* inf = info(sb);
       const int r = inf->r, h = inf->h, n_pos = min(inf->n_pos, NP);
-      MmaScal* sc = SC + ac * NP;
+      // SC[sb] is free: the producers reuse the v slot sb (and this unit's fullB[sb], waited
+      // above, completes) only after the epilogue of unit i - NB, the last reader, is done
+      MmaScal* sc = SC + sb * NP;
       float* DEC = DEC0 + db * (NP * UC);
       // position p = lane: beam, new record row, decay walk
       const int p = lane;
@@ -565,7 +567,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&dec_ready[db]);
-        mbar_arrive(&scal_ready[ac]);
+        mbar_arrive(&scal_ready[sb]);
       }
     }
   } else if (warp < kMmaWEpi) {
@@ -609,9 +611,8 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       }
       // c0_p = k_p . q_p for the epilogue (fp32 sums of the staged bf16 rows): thread
       // (p, quarter) of the 128 coefficient threads takes a quarter of the row, then the four
-      // partial sums are added across lanes; SC[ac] is free once the epilogue of unit i - NA is
-      // done.
-      if (i >= NA) ok = ok && mbar_wait_bounded(&acc_empty[ac], ((i - NA) / NA) & 1);
+      // partial sums are added across lanes; SC[sb] is free since fullB[sb] of this unit
+      // completed (the prep warp's comment says why).
       {
         const int tc = 32 * sp + lane, p = tc >> 2, qd = tc & 3;
         const unsigned char* xs = stage(s);
@@ -633,7 +634,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         }
         c0 += __shfl_xor_sync(kFull, c0, 1);
         c0 += __shfl_xor_sync(kFull, c0, 2);
-        if (qd == 0) SC[ac * NP + p].c0 = c0;
+        if (qd == 0) SC[sb * NP + p].c0 = c0;
         // append k_p (row block 0 only): the 128 threads copy the staged k rows (16-byte
         // chunks) into the records
         const int n_pos = inf->rb == 0 ? min(inf->n_pos, NP) : 0;
@@ -649,7 +650,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         }
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&scal_ready[ac]);
+          mbar_arrive(&scal_ready[sb]);
           mbar_arrive(&emptyA[s]);                   // done with the operand stage
         }
       }
@@ -726,13 +727,13 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     for (int i = 0; i < n_my; ++i) {
       const int sb = i % NB, ac = i % NA;
       bool ok = mbar_wait_bounded(&acc_full[ac], (i / NA) & 1);
-      ok = ok && mbar_wait_bounded(&scal_ready[ac], (i / NA) & 1);
+      ok = ok && mbar_wait_bounded(&scal_ready[sb], (i / NB) & 1);
       if (!__all_sync(kFull, ok)) {
         if (lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 26, t);
         break;
       }
       tc_fence_after();
-      const MmaScal* sc = SC + ac * NP;
+      const MmaScal* sc = SC + sb * NP;
       const unsigned char* Vb = vslot(sb);          // [2][32][128 B] sw128
       const MmaInfo* inf = info(sb);
       const int n_pos = min(inf->n_pos, NP), U = inf->U;
