@@ -192,14 +192,34 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t = a.t, n_anc = t - 1;
-  // walk items (request, head, row block), row block fastest, dealt round-robin: CTA c takes
+  // Walk items (request, head, row block), row block fastest, dealt round-robin: CTA c takes
   // items c, c + G, c + 2G, ... so that at any time the CTAs work on the row blocks and
   // neighbouring heads of the same beams (whose q, k, v, o rows and records lie next to each
-  // other in memory, and whose q / k rows a second row block finds in L2)
+  // other in memory, and whose q / k rows a second row block finds in L2). When items hold many
+  // units (4 or more on average), only the full rounds of G items are dealt that way: the units
+  // of the remaining items (the tail, items T0 .. n_items - 1, units in item order) are split
+  // into G contiguous ranges, one per CTA, so that the last round does not leave CTAs idle.
+  // Units in item order: item it of request r starts at unit H NRB uoff[r] + (it - r H NRB)
+  // ucnt[r].
   const int HN = a.H * NRB;
   const int n_items = a.R * HN;
-  int n_my = 0;
-  for (int it = blockIdx.x; it < n_items; it += gridDim.x) n_my += __ldcg(up.ucnt + it / HN);
+  const int GX = int(gridDim.x);
+  const bool split_tail = HN * __ldcg(up.uoff + a.R) >= 4 * n_items;
+  const int F = split_tail ? n_items / GX : (n_items + GX - 1) / GX;   // rounds dealt round-robin
+  const int T0 = split_tail ? F * GX : n_items;                         // first item of the tail
+  int tail_begin = 0, n_tail = 0;
+  if (T0 < n_items) {
+    const int r0 = T0 / HN;
+    const int U0 = HN * __ldcg(up.uoff + r0) + (T0 - r0 * HN) * __ldcg(up.ucnt + r0);
+    const int NT = HN * __ldcg(up.uoff + a.R) - U0;
+    tail_begin = U0 + int((long long)NT * blockIdx.x / GX);
+    n_tail = U0 + int((long long)NT * (blockIdx.x + 1) / GX) - tail_begin;
+  }
+  int n_my = n_tail;
+  for (int f = 0; f < F; ++f) {
+    const int it = int(blockIdx.x) + f * GX;
+    if (it < T0) n_my += __ldcg(up.ucnt + it / HN);
+  }
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -241,9 +261,26 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     // ------------------------------------------------------------------ producers
     const int pw = warp < kMmaWMma ? warp : warp - 1;     // 0..4
     int issued = 0;
+    // the item and unit holding global unit index u (item-major order)
+    auto locate = [&](int u, int& it_, int& r_, int& k_) {
+      int lo = 0, hi = a.R - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (HN * __ldcg(up.uoff + mid) <= u) lo = mid;
+        else hi = mid - 1;
+      }
+      r_ = lo;
+      const int c_ = __ldcg(up.ucnt + lo);
+      const int rem = u - HN * __ldcg(up.uoff + lo);
+      it_ = lo * HN + rem / c_;
+      k_ = rem % c_;
+    };
     if (n_my > 0) {
-      int it = int(blockIdx.x), k = 0;
-      int r = it / HN, h = (it / NRB) % a.H, rb = it % NRB;
+      int it = int(blockIdx.x), k = 0, r = 0;
+      bool tail = F == 0;
+      if (tail) locate(tail_begin, it, r, k);
+      r = it / HN;
+      int h = (it / NRB) % a.H, rb = it % NRB;
       int cnt = __ldcg(up.ucnt + r);
       const int* rec = up.urec + (size_t(r) * up.maxU + k) * kUnitRecInts;
       int x0 = __ldcg(rec + lane), x1 = __ldcg(rec + 32 + lane), x2 = __ldcg(rec + 64 + lane);
@@ -258,9 +295,19 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         }
         // the next unit of the walk; its record is fetched now and used in the next iteration
         int nit = it, nr = r, nh = h, nrb = rb, nk = k + 1, ncnt = cnt;
+        bool ntail = tail;
         if (nk == cnt) {
           nk = 0;
-          nit = it + int(gridDim.x);
+          if (tail) {
+            nit = it + 1;
+          } else {
+            nit = it + GX;
+            if (nit >= T0 && n_tail > 0) {
+              int rr;
+              locate(tail_begin, nit, rr, nk);
+              ntail = true;
+            }
+          }
           nr = nit / HN;
           nh = (nit / NRB) % a.H;
           nrb = nit % NRB;
@@ -280,7 +327,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
           // ahead of the coefficient warps' loads: 2 x DVB rows x 2 d_k bytes
           const int npf = (prev_it < 0 ? 2 : 1);
           for (int q = 0; q < npf; ++q) {
-            const int iq = it + (npf == 2 ? q : 1) * int(gridDim.x);
+            const int iq = (tail || it + GX >= T0) ? it + (npf == 2 ? q : 1) : it + (npf == 2 ? q : 1) * GX;
             if (iq < n_items) {
               const size_t row0 = size_t(iq / NRB) * MP + size_t(iq % NRB) * 128;
               const unsigned char* hi_b = reinterpret_cast<const unsigned char*>(S_hi + row0 * DK);
@@ -405,6 +452,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
         x1 = y1;
         x2 = y2;
         it = nit;
+        tail = ntail;
         r = nr;
         h = nh;
         rb = nrb;
