@@ -382,6 +382,11 @@ def bench_workload(w: wl.Workload, args, ctx) -> dict:
             if evs is not None:
                 evs[t][1].record(stream)
 
+    def decode_on(dec, st):
+        # the same decode with `st` as the current stream (every call takes the current stream)
+        with torch.cuda.stream(st):
+            decode(dec)
+
     # the tensor-core path takes bf16 inputs and widths 64, 128, 256; other workloads (the tiny
     # fp32 one) decode on the fp32 replay path
     tensor = tensor_path_ok(w)
@@ -395,15 +400,42 @@ def bench_workload(w: wl.Workload, args, ctx) -> dict:
         raise RuntimeError(f"device error during warm-up: {ola.ola_strerror(st)}")
 
     K = args.steps
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(w.T)]
-           for _ in range(K)]
+    # One bench step = one whole decode. By default the decode (ola_reset + T ola_step calls,
+    # issued through the C ABI on a side stream) is recorded once into a CUDA graph and the timed
+    # region replays it K times, so that the host's per-call work (argument checks, tensor maps,
+    # launches) is not on the device timeline; every kernel of every step still runs.
+    graph, timing = None, "eager: K decodes issued through the C ABI"
+    if not args.no_graph:
+        try:
+            cap = torch.cuda.Stream(device=dev)
+            cap.wait_stream(stream)
+            with torch.cuda.stream(cap):
+                decode_on(dec, cap)               # the handle's last stream becomes `cap`
+            cap.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=cap):
+                decode_on(dec, cap)
+            graph.replay()
+            torch.cuda.synchronize()
+            if dec.error() != ola.OLA_OK:
+                raise RuntimeError("device error in the captured decode")
+            timing = ("CUDA graph of one whole decode (ola_reset + T ola_step calls through the "
+                      "C ABI), replayed K times")
+        except Exception as ex:                   # capture not possible: time eagerly
+            graph = None
+            timing = f"eager (graph capture failed: {type(ex).__name__})"
+            torch.cuda.synchronize()
+            dec.reset()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier()
         torch.cuda.synchronize()
         e0.record(stream)
         for k in range(K):
-            decode(dec, evs[k])
+            if graph is not None:
+                graph.replay()
+            else:
+                decode(dec)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -412,9 +444,16 @@ def bench_workload(w: wl.Workload, args, ctx) -> dict:
     if st != ola.OLA_OK:
         raise RuntimeError(f"device error in the timed region: {ola.ola_strerror(st)}")
     ms = max_ranks(e0.elapsed_time(e1))
+    # per-step breakdown (not the metric): eager decodes with CUDA events around every ola_step
+    K2 = min(K, 20)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(w.T)]
+           for _ in range(K2)]
+    for k in range(K2):
+        decode(dec, evs[k])
+    torch.cuda.synchronize()
     step_ms = np.array([[evs[k][t][0].elapsed_time(evs[k][t][1]) for t in range(w.T)]
-                        for k in range(K)])
-    per_launch_ms = step_ms.mean(axis=0)               # ola_step t, averaged over K
+                        for k in range(K2)])
+    per_launch_ms = step_ms.mean(axis=0)               # ola_step t, averaged over K2
     units_per_step = w.R * w.H * w.B * w.T
     value = job_value(world, units_per_step, K, ms)
 
@@ -422,7 +461,9 @@ def bench_workload(w: wl.Workload, args, ctx) -> dict:
     peaks = measured_peaks()
     bytes_t = algorithmic_bytes_per_step(w, parents)
     lit_t = state_and_record_bytes_per_step(w, parents)
-    achieved = sum(bytes_t) / (per_launch_ms.sum() / 1e3) / 1e9
+    # one decode's algorithmic bytes over its device time in the timed region (plan kernels
+    # included)
+    achieved = sum(bytes_t) / (ms / K / 1e3) / 1e9
     flops = tensor_flops_per_step(w) * w.T
     tensor_time = flops / (peaks["bf16_tflops"] * 1e12) if tensor else 0.0
     hbm_time = sum(bytes_t) / (peaks["hbm_gbs"] * 1e9)
@@ -432,10 +473,11 @@ def bench_workload(w: wl.Workload, args, ctx) -> dict:
                 "kernel": "ola_step = " + (replay_kernel_label(w) if tensor else
                                            "ola::replay_simt_kernel"),
                 "algorithmic_bytes_per_decode": int(sum(bytes_t)),
-                "frac_state_and_records_only": sum(lit_t) / (per_launch_ms.sum() / 1e3) / 1e9 /
+                "frac_state_and_records_only": sum(lit_t) / (ms / K / 1e3) / 1e9 /
                                                peaks["hbm_gbs"],
                 "algorithmic_bytes_per_launch": [int(b) for b in bytes_t],
-                "launch_ms": [round(float(x), 4) for x in per_launch_ms],
+                "launch_ms_eager": [round(float(x), 4) for x in per_launch_ms],
+                "timed_over": "one decode of the timed region (K graph replays / K)",
                 "t_roof_ms": 1e3 * max(tensor_time, hbm_time),
                 "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"}
 
@@ -453,7 +495,8 @@ def bench_workload(w: wl.Workload, args, ctx) -> dict:
                                 "no flush: each decode step streams %.0f MB, inside the 126 MB "
                                 "L2 (a small configuration; its time is launch- and "
                                 "latency-bound)" % (max(bytes_t) / 1e6)),
-                         "parallelism": f"replicas x{world} (requests sharded, no collective)"},
+                         "parallelism": f"replicas x{world} (requests sharded, no collective)",
+                         "timing": timing},
               "roofline": roofline, "clocks": clocks,
               "gpu_launches": (2 if tensor else 1) * w.T * K}
 
@@ -702,6 +745,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-compare", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eagerly issued decodes instead of CUDA-graph replays")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--requests", type=int, default=0,

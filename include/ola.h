@@ -75,10 +75,10 @@ enum { OLA_PATH_REPLAY = 0, OLA_PATH_FULLSTATE = 1, OLA_PATH_REPLAYSSM = 2 };
 /* how the contractions of the replay path are computed:
  * FP32 = CUDA-core fp32 FMA everywhere; TENSOR = tcgen05 tensor cores, bf16 operands with
  * S_ctx split into a bf16 high part and a bf16 remainder (two MMAs, fp32 accumulate in
- * tensor memory). With d_v = 128, d_k in {64, 128}, B <= 1024 and T_max <= 12 the replay
- * accumulation over the ancestor records also runs on tensor cores: the records' w rows are
- * then kept as a bf16 high part and a bf16 remainder (same bytes as fp32) and each product
- * runs as three bf16 MMAs with fp32 accumulation; otherwise it runs in fp32 on CUDA cores. */
+ * tensor memory). With B <= 1024 and T_max <= 12 the replay accumulation over the ancestor
+ * records also runs on tensor cores: the records' w rows are then kept as a bf16 high part and
+ * a bf16 remainder (same bytes as fp32) and each product runs as three bf16 MMAs with fp32
+ * accumulation; beyond those limits it runs in fp32 on CUDA cores. */
 enum { OLA_MATH_FP32 = 0, OLA_MATH_TENSOR = 1 };
 
 typedef struct {

@@ -8,9 +8,45 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "ola.h"
 
 namespace ola {
+
+// Host: runs `fn` (a kernel attribute setting, a device query) on the first call for each device
+// and remembers that it succeeded, so that per-step launches skip it. Thread-safe; `done` holds
+// one bit per device (devices past 63 always run `fn`).
+template <typename F>
+inline cudaError_t once_per_device(std::atomic<uint64_t>& done, F fn) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return fn();
+  const uint64_t bit = uint64_t(1) << dev;
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = fn();
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+// Host: number of SMs of the current device (queried once per device).
+inline cudaError_t device_sm_count(int* n) {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_acquire);
+    if (c > 0) {
+      *n = c;
+      return cudaSuccess;
+    }
+  }
+  e = cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) cache[dev].store(*n, std::memory_order_release);
+  return e;
+}
 
 // Everything one decode step needs. Record storage (the transition records of every beam,
 // appended once and never moved; the history-replay path keeps v_t and beta_t instead of w_t):

@@ -437,8 +437,19 @@ __global__ void __launch_bounds__(512) plan_units_kernel(StepArgs a, UnitPlan up
 
 cudaError_t launch_plan_units(const StepArgs& a, const UnitPlan& up, cudaStream_t stream) {
   const size_t smem = plan_units_smem(a.B, a.T_max);
-  cudaError_t e = cudaFuncSetAttribute(plan_units_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  // the attribute is a limit, set once per device to the largest a handle may need (handles
+  // whose plan needs more than the device offers are refused at create)
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = once_per_device(configured, [] {
+    int dev = 0, optin = 0;
+    cudaError_t x = cudaGetDevice(&dev);
+    if (x == cudaSuccess)
+      x = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (x == cudaSuccess)
+      x = cudaFuncSetAttribute(plan_units_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               optin);
+    return x;
+  });
   if (e != cudaSuccess) return e;
   plan_units_kernel<<<a.R, 512, smem, stream>>>(a, up);
   return cudaGetLastError();

@@ -909,8 +909,10 @@ static cudaError_t launch_mma_t(const void* S_hi, const void* S_lo, const StepAr
                                 cudaStream_t stream) {
   const MmaLayout L = mma_layout_of<DK, DV>();
   auto kern = replay_mma_kernel<DK, DV>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(L.bytes));
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = once_per_device(configured, [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(L.bytes));
+  });
   if (e != cudaSuccess) return e;
   kern<<<n_sm, kMmaWarps * 32, L.bytes, stream>>>(static_cast<const __nv_bfloat16*>(S_hi),
                                                   static_cast<const __nv_bfloat16*>(S_lo), a, up,
@@ -933,9 +935,8 @@ cudaError_t launch_replay_mma(const StepArgs& a, const UnitPlan& up, const void*
     return cudaErrorInvalidValue;
   cudaError_t e = launch_plan_units(a, up, stream);
   if (e != cudaSuccess) return e;
-  int dev = 0, n_sm = 0;
-  e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  int n_sm = 0;
+  e = device_sm_count(&n_sm);
   if (e != cudaSuccess) return e;
 #define OLA_MMA_CASE(DK_, DV_)                                                              \
   case DK_ * 1000 + DV_:                                                                    \
