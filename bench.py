@@ -337,6 +337,31 @@ def run_ours(args):
     return 0
 
 
+def capture_decode(torch, ola, dec, decode, stream):
+    """Record one call of `decode` (ola_reset + T ola_step calls through the C ABI, taking the
+    current stream) into a CUDA graph on a side stream. Returns (graph, note); graph is None if
+    the capture failed here, and the caller then issues decodes eagerly."""
+    try:
+        cap = torch.cuda.Stream(device=stream.device)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            decode(dec)                           # the handle's last stream becomes `cap`
+        cap.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            decode(dec)
+        graph.replay()
+        torch.cuda.synchronize()
+        if dec.error() != ola.OLA_OK:
+            raise RuntimeError("device error in the captured decode")
+        return graph, ("CUDA graph of one whole decode (ola_reset + T ola_step calls through the "
+                       "C ABI), replayed K times")
+    except Exception as ex:                       # noqa: BLE001 - report and time eagerly
+        torch.cuda.synchronize()
+        dec.reset()
+        return None, f"eager (graph capture failed: {type(ex).__name__})"
+
+
 def tensor_path_ok(w: wl.Workload) -> bool:
     return w.dtype == "bf16" and w.d_k in (64, 128, 256) and w.d_v in (64, 128, 256)
 
@@ -382,11 +407,6 @@ def bench_workload(w: wl.Workload, args, ctx) -> dict:
             if evs is not None:
                 evs[t][1].record(stream)
 
-    def decode_on(dec, st):
-        # the same decode with `st` as the current stream (every call takes the current stream)
-        with torch.cuda.stream(st):
-            decode(dec)
-
     # the tensor-core path takes bf16 inputs and widths 64, 128, 256; other workloads (the tiny
     # fp32 one) decode on the fp32 replay path
     tensor = tensor_path_ok(w)
@@ -406,26 +426,7 @@ def bench_workload(w: wl.Workload, args, ctx) -> dict:
     # launches) is not on the device timeline; every kernel of every step still runs.
     graph, timing = None, "eager: K decodes issued through the C ABI"
     if not args.no_graph:
-        try:
-            cap = torch.cuda.Stream(device=dev)
-            cap.wait_stream(stream)
-            with torch.cuda.stream(cap):
-                decode_on(dec, cap)               # the handle's last stream becomes `cap`
-            cap.synchronize()
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph, stream=cap):
-                decode_on(dec, cap)
-            graph.replay()
-            torch.cuda.synchronize()
-            if dec.error() != ola.OLA_OK:
-                raise RuntimeError("device error in the captured decode")
-            timing = ("CUDA graph of one whole decode (ola_reset + T ola_step calls through the "
-                      "C ABI), replayed K times")
-        except Exception as ex:                   # capture not possible: time eagerly
-            graph = None
-            timing = f"eager (graph capture failed: {type(ex).__name__})"
-            torch.cuda.synchronize()
-            dec.reset()
+        graph, timing = capture_decode(torch, ola, dec, decode, stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier()
@@ -638,7 +639,8 @@ def fullstate_bytes_per_step(w: wl.Workload, parents: np.ndarray) -> list:
 def run_sweep(args):
     """The operator sweep: nine (d_k, d_v) geometries x request counts x beam widths x decode
     lengths (405 shapes), H = 16 heads, bf16 inputs, Zipf(1.0) parents, a shared state from a
-    1K-token prompt. Per shape: replay (tensor path) and FullState time per decode, capacity
+    1K-token prompt. Per shape: replay (tensor path) and FullState time per decode (CUDA-graph
+    replays of one decode, as in the bench; --no-graph for eager calls), capacity
     bytes, algorithmic DRAM bytes and the fraction of the measured HBM bandwidth, and the
     largest |o| difference between the two paths. One JSON line per shape."""
     import torch
@@ -656,22 +658,29 @@ def run_sweep(args):
     stream = torch.cuda.current_stream()
 
     def timed(dec, steps, par, outs, reps, warm):
-        def decode():
-            dec.reset()
+        def decode(d):
+            d.reset()
             for t in range(len(steps)):
                 s = steps[t]
-                dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], par[t], out=outs[t])
+                d.step(s["q"], s["k"], s["v"], s["g"], s["beta"], par[t], out=outs[t])
         for _ in range(warm):
-            decode()
+            decode(dec)
         torch.cuda.synchronize()
+        graph = None
+        if not args.no_graph and reps > 0:
+            graph, _ = capture_decode(torch, ola, dec, decode, stream)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(reps):
-            decode()
+            if graph is not None:
+                graph.replay()
+            else:
+                decode(dec)
         b.record(stream)
         torch.cuda.synchronize()
         if dec.error() != ola.OLA_OK:
             raise RuntimeError(f"device error: {ola.ola_strerror(dec.error())}")
+        del graph
         return a.elapsed_time(b) / max(reps, 1)
 
     for dk, dv in geoms:
