@@ -452,3 +452,23 @@ def test_compact_requests_converging_at_different_steps(path):
     err = max_abs(o, ref)
     assert err <= tol_for(path), (path, err)
     assert np.array_equal(anc, oracle.ancestry_table(parents)[:, :, base:])
+
+
+@pytest.mark.parametrize("R,H,d_v", [(37, 4, 128), (149, 1, 128), (3, 16, 256), (5, 61, 64)])
+def test_walk_item_counts(R, H, d_v):
+    """The tensor-core replay deals its (request, head, row block) items to the 148 CTAs in
+    round-robin rounds and splits the units of a last, partial round into contiguous ranges:
+    exactly one round (148 items), one round plus one item (149), row-blocked items (d_v = 256:
+    96 items, all in the split tail) and 305 items (two rounds plus a tail). Sampled units
+    include the last items of the walk; ancestry is compared in full."""
+    w = wl.WORKLOADS["single_request"].scaled(R=R, H=H, d_k=64, d_v=d_v, B=130, P=16, T=3)
+    S32, steps, dev_steps, parents = small_problem(w)
+    n = R * H
+    units = sorted({(u // H, u % H) for u in [0, 1, n // 2, n - 3, n - 2, n - 1]})
+    ref = oracle_outputs(S32, steps, parents, units=units)
+    o, anc, status = run_library(S32.cuda(), dev_steps, parents, "replay_tensor", w.torch_dtype)
+    assert status == ola.OLA_OK
+    err = max_abs(o, ref)
+    print(f"walk R={R} H={H} d_v={d_v}: max-abs {err:.3e}")
+    assert err <= tol_for("replay_tensor")
+    assert np.array_equal(anc, oracle.ancestry_table(parents))
