@@ -184,7 +184,9 @@ ola_status ola_get_error(ola_handle h);
  * path the folded records are raw tokens and are applied with the gated delta rule itself.
  *   out_folded : host int32, optional (NULL): number of folded steps (0 if none).
  * Synchronises `stream`, which must be the stream of the handle's previous calls (or ordered
- * after them). FullState handles hold no records: nothing is folded.
+ * after them). FullState handles keep every beam's state, so nothing is folded there: only the
+ * ancestry rows of the shared slots are dropped and t lowered, which lets them decode past T_max
+ * too (out_folded counts those slots).
  * Errors: INVALID_ARG (NULL handle), the sticky device error, CUDA. */
 ola_status ola_compact(ola_handle h, int32_t* out_folded, void* stream);
 

@@ -171,7 +171,7 @@ Sizes sizes_of(const ola_geometry* g) {
   z.rank = g->math == OLA_MATH_TENSOR ? 2 * R * B * 4 : 0;
   z.pchain = g->math == OLA_MATH_TENSOR ? R * B * T * 4 : 0;
   z.err = 16;
-  z.lens = g->path != OLA_PATH_FULLSTATE ? R * 4 : 0;
+  z.lens = R * 4;
   if (uses_mma(g)) {
     z.ucnt = R * 4;
     z.uoff = (R + 1) * 4;
@@ -513,7 +513,7 @@ ola_status ola_compact(ola_handle h, int32_t* out_folded, void* stream) {
   if (h->sticky) return static_cast<ola_status>(h->sticky);
   const ola_geometry& g = h->g;
   const int t = h->t;
-  if (g.path == OLA_PATH_FULLSTATE || t < 2) return OLA_OK;   // nothing to fold
+  if (t < 2) return OLA_OK;   // nothing to fold
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;
   // shared chain prefix of every request (into the handle's own buffer: nothing is allocated)
@@ -526,6 +526,16 @@ ola_status ola_compact(ola_handle h, int32_t* out_folded, void* stream) {
   int c = t - 1;
   for (int x : host) c = std::min(c, x);
   if (c <= 0) return OLA_OK;
+  if (g.path == OLA_PATH_FULLSTATE) {
+    // the beams' states are materialised and hold every step: only the ancestry rows of the
+    // shared slots are dropped; the state buffers follow the parity of the lowered step count
+    e = launch_chain_shift(h->C, g.R, g.B, g.T_max, t, c, st);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (c & 1) std::swap(h->FS[0], h->FS[1]);
+    h->t = t - c;
+    if (out_folded) *out_folded = c;
+    return OLA_OK;
+  }
   // fold the shared records into S_ctx (and its bf16 split), then move the later record slots
   // and the chain rows down by c
   const bool rss = g.path == OLA_PATH_REPLAYSSM;

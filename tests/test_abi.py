@@ -66,7 +66,7 @@ def test_workspace_bytes_formula(L):
               T * R * H * B * 4 + T * R * B * T * 4 + 16 + R * 4)
     assert ola.ola_workspace_bytes(g) == expect
     gf = _geom(R=2, H=3, d_k=64, d_v=128, B=40, T_max=5, path=ola.OLA_PATH_FULLSTATE)
-    expect_fs = R * H * dv * dk * 4 + 2 * R * H * B * dv * dk * 4 + T * R * B * T * 4 + 16
+    expect_fs = R * H * dv * dk * 4 + 2 * R * H * B * dv * dk * 4 + T * R * B * T * 4 + 16 + R * 4
     assert ola.ola_workspace_bytes(gf) == expect_fs
     # history-replay path: the raw tokens of every record (k, v in the input dtype, alpha,
     # beta), no w records and no per-beam state

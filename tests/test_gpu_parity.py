@@ -347,7 +347,7 @@ def _converging_parents(w, merge_steps):
     return par
 
 
-@pytest.mark.parametrize("path", ["replay_tensor", "replay_fp32", "replayssm"])
+@pytest.mark.parametrize("path", ["replay_tensor", "replay_fp32", "replayssm", "fullstate"])
 def test_compact_decodes_past_t_max(path):
     """A decode of 8 steps on a handle of T_max = 4: ola_compact after steps 3 and 6 folds the
     chain slots every beam shares into S_ctx, and the outputs of every step still match the
@@ -415,7 +415,7 @@ def _shared_prefix(table):
     return table.shape[1]
 
 
-@pytest.mark.parametrize("path", ["replay_tensor", "replay_fp32", "replayssm"])
+@pytest.mark.parametrize("path", ["replay_tensor", "replay_fp32", "replayssm", "fullstate"])
 def test_compact_requests_converging_at_different_steps(path):
     """Three requests whose beams converge at different steps (each request's own merges), a
     handle of T_max = 4 decoding 9 steps with ola_compact after every step: each call folds the
