@@ -348,7 +348,7 @@ def capture_decode(torch, ola, dec, decode, stream):
             decode(dec)                           # the handle's last stream becomes `cap`
         cap.synchronize()
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=cap):
+        with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
             decode(dec)
         graph.replay()
         torch.cuda.synchronize()

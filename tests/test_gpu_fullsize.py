@@ -98,7 +98,8 @@ def _tail_units(w, n=N_SM):
 def test_stress_full_size(pool):
     w = wl.WORKLOADS["stress"]
     units = [(0, 0), (0, 1), (1, 7), (37, 9)] + _tail_units(w)
-    _run(w, ["replay_tensor", "replay_fp32"], units, pool)
+    # the two comparison paths too (FullState holds 2 x 34 GB of per-beam states here)
+    _run(w, ["replay_tensor", "replay_fp32", "fullstate", "replayssm"], units, pool)
 
 
 def test_multi_request_full_size_all_paths(pool):
