@@ -714,42 +714,40 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
       }
       tc_fence_after();
       if (U > 0) {
-        // Cf = DEC * G, written as bf16 hi + lo, 16 records at a time. Thread n = 16 sp + lane
-        // (lanes 0-15) holds row n of G (the M = 64 layout puts rows 16 sp .. 16 sp + 15 in
-        // lanes 0-15 of subpartition sp).
+        // Cf = DEC * G, written as bf16 hi + lo, 16 records at a time. Lanes 0-15 hold rows
+        // n = 16 sp + lane of G (the M = 64 layout puts rows 16 sp .. 16 sp + 15 in lanes 0-15 of
+        // subpartition sp); lanes 16-31 take over records 8-15 of the same rows, so that every
+        // lane converts and stores one 8-record chunk.
         const uint32_t tg = tmem + (uint32_t(32 * sp) << 16) + uint32_t(ac) * 128u + 64u;
-        const int nrow = 16 * sp + (lane & 15), p = nrow & 31;
+        const int nrow = 16 * sp + (lane & 15), p = nrow & 31, q2 = lane >> 4;
         const float* dr = DEC0 + db * (NP * UC) + p * UC;
 #pragma unroll 1
         for (int h16 = 0; h16 < UC / 16; ++h16) {
           if (16 * h16 >= U) break;                   // warp-uniform
           float gr[16];
           tmem_ld16(tg + 16u * h16, gr);
-          if (lane < 16) {
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-              const int q = 2 * h16 + q2;
-              const float4 d0 = *reinterpret_cast<const float4*>(dr + 8 * q);
-              const float4 d1 = *reinterpret_cast<const float4*>(dr + 8 * q + 4);
-              const float v[8] = {gr[8 * q2] * d0.x,     gr[8 * q2 + 1] * d0.y,
-                                  gr[8 * q2 + 2] * d0.z, gr[8 * q2 + 3] * d0.w,
-                                  gr[8 * q2 + 4] * d1.x, gr[8 * q2 + 5] * d1.y,
-                                  gr[8 * q2 + 6] * d1.z, gr[8 * q2 + 7] * d1.w};
-              uint32_t hw[4], lw[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat162 hi2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-                const float2 hf2 = __bfloat1622float2(hi2);
-                const __nv_bfloat162 lo2 =
-                    __floats2bfloat162_rn(v[2 * e] - hf2.x, v[2 * e + 1] - hf2.y);
-                hw[e] = *reinterpret_cast<const uint32_t*>(&hi2);
-                lw[e] = *reinterpret_cast<const uint32_t*>(&lo2);
-              }
-              const uint32_t off = uint32_t(nrow) * 128u + uint32_t((q ^ (nrow & 7)) << 4);
-              *reinterpret_cast<uint4*>(CH + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-              *reinterpret_cast<uint4*>(CL + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            }
+          for (int e = 0; e < 8; ++e) {
+            const float lv = __shfl_up_sync(kFull, gr[8 + e], 16);
+            if (lane >= 16) gr[e] = lv;
           }
+          const int q = 2 * h16 + q2;
+          const float4 d0 = *reinterpret_cast<const float4*>(dr + 8 * q);
+          const float4 d1 = *reinterpret_cast<const float4*>(dr + 8 * q + 4);
+          const float v[8] = {gr[0] * d0.x, gr[1] * d0.y, gr[2] * d0.z, gr[3] * d0.w,
+                              gr[4] * d1.x, gr[5] * d1.y, gr[6] * d1.z, gr[7] * d1.w};
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 hi2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+            const float2 hf2 = __bfloat1622float2(hi2);
+            const __nv_bfloat162 lo2 = __floats2bfloat162_rn(v[2 * e] - hf2.x, v[2 * e + 1] - hf2.y);
+            hw[e] = *reinterpret_cast<const uint32_t*>(&hi2);
+            lw[e] = *reinterpret_cast<const uint32_t*>(&lo2);
+          }
+          const uint32_t off = uint32_t(nrow) * 128u + uint32_t((q ^ (nrow & 7)) << 4);
+          *reinterpret_cast<uint4*>(CH + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(CL + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
         fence_proxy_async_smem();
       }
