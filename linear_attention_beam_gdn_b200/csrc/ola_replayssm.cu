@@ -25,9 +25,11 @@
 // decode 1.3x slower).
 //
 // Grid: (request, head) x blocks of state rows. A CTA of 8 warps holds its rows of S_ctx in
-// shared memory (read from HBM once per step and CTA) and walks every beam of the request;
-// each warp owns RPW rows and rebuilds them beam after beam, reading the chain's keys through
-// L2, one ancestor ahead. fp32 arithmetic on CUDA cores throughout.
+// shared memory (read from HBM once per step and CTA) and walks every beam of the request,
+// grouped by parent (a counting sort of the parents); each warp owns RPW rows and rebuilds
+// them over the parent's chain once per parent, reading the chain's keys through L2 one
+// ancestor ahead, keeps that state in shared memory and applies each child's own token to it.
+// Nothing survives the step. fp32 arithmetic on CUDA cores throughout.
 #include "ola_device.cuh"
 
 namespace ola {
@@ -44,9 +46,15 @@ struct RsShape {
   static constexpr int V4 = EL / 4;                    // float4 per lane
 };
 
+// shared memory: S_ctx slices and the rebuilt parent state ([V4][kRsThreads] float4 each), then
+// the beams grouped by parent and the counts of the sort ([B] int each)
 template <int DK>
-__host__ __device__ constexpr size_t rs_smem_bytes() {
+__host__ __device__ constexpr size_t rs_state_bytes() {
   return size_t(kRsThreads) * RsShape<DK>::EL * 4;
+}
+template <int DK>
+__host__ __device__ constexpr size_t rs_smem_bytes(int B) {
+  return 2 * rs_state_bytes<DK>() + 2 * size_t(B) * 4;
 }
 
 // EL consecutive inputs starting at element `e0` of row `row` of a [.., DK] array, widened
@@ -81,6 +89,12 @@ __device__ __forceinline__ void load_slice(float (&x)[EL], const void* base, siz
   }
 }
 
+// Parent of beam b as the append pass reads it (out of range: 0; the append pass reports it).
+__device__ __forceinline__ int clamped_parent(const StepArgs& a, int r, int b) {
+  const int p = a.parent[size_t(r) * a.B + b];
+  return ((a.t == 1 && p != 0) || p < 0 || p >= a.B) ? 0 : p;
+}
+
 // One transition of the lane's slice of row i, the row held as sigma * S^:
 // u = sigma (S^_i . k) (over the LPR lanes of the row), w = beta (v_i - alpha u),
 // S_i <- alpha S_i + w k, i.e. sigma <- alpha sigma, S^_i += (w / sigma) k.
@@ -112,6 +126,9 @@ replayssm_kernel(StepArgs a) {
   static_assert(EL % 8 == 0, "a lane's slice is whole 16-byte vectors");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float4* S0 = reinterpret_cast<float4*>(smem_raw);      // [V4][kRsThreads]: S_ctx slices
+  float4* SP = S0 + V4 * kRsThreads;                     // the rebuilt state of the current parent
+  int* ord = reinterpret_cast<int*>(SP + V4 * kRsThreads);   // [B] beams grouped by parent
+  int* cnt = ord + a.B;                                       // [B] counts, then offsets
 
   const int rh = blockIdx.x;
   const int r = rh / a.H, h = rh % a.H;
@@ -160,57 +177,97 @@ replayssm_kernel(StepArgs a) {
       }
     }
   }
+  // 3. the beams grouped by parent: a counting sort of the (clamped) parents; the order within
+  //    a group does not matter (every child of a parent starts from the same rebuilt state)
+  for (int b = tid; b < a.B; b += kRsThreads) cnt[b] = 0;
+  __syncthreads();
+  for (int b = tid; b < a.B; b += kRsThreads) atomicAdd(&cnt[clamped_parent(a, r, b)], 1);
+  __syncthreads();
+  if (warp == 0) {                                       // exclusive scan of the counts
+    int carry = 0;
+    for (int base = 0; base < a.B; base += 32) {
+      const int x = base + lane < a.B ? cnt[base + lane] : 0;
+      int y = x;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int z = __shfl_up_sync(0xffffffffu, y, off);
+        if (lane >= off) y += z;
+      }
+      if (base + lane < a.B) cnt[base + lane] = carry + y - x;
+      carry += __shfl_sync(0xffffffffu, y, 31);
+    }
+  }
+  __syncthreads();
+  for (int b = tid; b < a.B; b += kRsThreads) ord[atomicAdd(&cnt[clamped_parent(a, r, b)], 1)] = b;
   __syncthreads();
 
-  // 3. every beam of the request: rebuild this warp's rows from S_ctx along the parent's chain,
-  //    apply the beam's own token, project onto q_t
-  for (int b = 0; b < a.B; ++b) {
-    int p = a.parent[size_t(r) * a.B + b];
-    if ((t == 1 && p != 0) || p < 0 || p >= a.B) p = 0;   // reported by the append pass
-    int cidx = 0;
-    if (lane < n_anc) cidx = __ldg(a.C + chain_row(a, t - 2, r, p) + lane);
-
+  // 4. every beam of the request, a parent's children in a row: rebuild this warp's rows from
+  //    S_ctx along the parent's chain once per parent (kept in SP), apply the beam's own token,
+  //    project onto q_t
+  int prev_p = -1;
+  float sigma_p = 1.f;
+  for (int ib = 0; ib < a.B; ++ib) {
+    const int b = ord[ib];
+    const int p = clamped_parent(a, r, b);
     float S[EL];
-#pragma unroll
-    for (int j = 0; j < V4; ++j) {
-      const float4 f = S0[j * kRsThreads + tid];
-      S[4 * j] = f.x;
-      S[4 * j + 1] = f.y;
-      S[4 * j + 2] = f.z;
-      S[4 * j + 3] = f.w;
-    }
     float kc[EL], kn[EL];
     float vc = 0.f, ac = 1.f, bc = 0.f, sigma = 1.f;
     const size_t in = (size_t(r) * a.B + b) * a.H + h;
-    // the key, value and scalars of chain position j (j == n_anc: the beam's own token)
-    auto fetch = [&](int j, float (&kx)[EL], float& vx, float& ax, float& bx) {
-      const int c = __shfl_sync(0xffffffffu, cidx, j < n_anc ? j : 0);
-      if (j < n_anc) {
+    if (p != prev_p) {
+      // the parent's state: S_ctx, then the tokens of its chain
+      int cidx = 0;
+      if (lane < n_anc) cidx = __ldg(a.C + chain_row(a, t - 2, r, p) + lane);
+#pragma unroll
+      for (int j = 0; j < V4; ++j) {
+        const float4 f = S0[j * kRsThreads + tid];
+        S[4 * j] = f.x;
+        S[4 * j + 1] = f.y;
+        S[4 * j + 2] = f.z;
+        S[4 * j + 3] = f.w;
+      }
+      auto fetch = [&](int j, float (&kx)[EL], float& vx, float& ax, float& bx) {
+        const int c = __shfl_sync(0xffffffffu, cidx, j);
         const size_t rec = rec_index(a, j, r, h, c);
         load_slice<TIn, EL>(kx, a.Kr, rec, e0, DK);
         vx = row_ok ? to_f32(static_cast<const TIn*>(a.Vr)[rec * a.d_v + row]) : 0.f;
         ax = __ldg(a.A + rec);
         bx = __ldg(a.Br + rec);
-      } else {
-        load_slice<TIn, EL>(kx, a.k, in, e0, DK);
-        vx = row_ok ? to_f32(static_cast<const TIn*>(a.v)[in * size_t(a.d_v) + row]) : 0.f;
-        ax = expf(__ldg(a.g + in));
-        bx = __ldg(a.beta + in);
-      }
-    };
-    fetch(0, kc, vc, ac, bc);
-    for (int j = 0; j <= n_anc; ++j) {
-      float vn = 0.f, an = 1.f, bn = 0.f;
-      if (j < n_anc) fetch(j + 1, kn, vn, an, bn);   // one position ahead
-      rs_transition<EL, LPR>(S, sigma, kc, vc, ac, bc);
-      if (j < n_anc) {
+      };
+      if (n_anc > 0) fetch(0, kc, vc, ac, bc);
+      for (int j = 0; j < n_anc; ++j) {
+        float vn = 0.f, an = 1.f, bn = 0.f;
+        if (j + 1 < n_anc) fetch(j + 1, kn, vn, an, bn);   // one position ahead
+        rs_transition<EL, LPR>(S, sigma, kc, vc, ac, bc);
+        if (j + 1 < n_anc) {
 #pragma unroll
-        for (int e = 0; e < EL; ++e) kc[e] = kn[e];
-        vc = vn;
-        ac = an;
-        bc = bn;
+          for (int e = 0; e < EL; ++e) kc[e] = kn[e];
+          vc = vn;
+          ac = an;
+          bc = bn;
+        }
       }
+#pragma unroll
+      for (int j = 0; j < V4; ++j)
+        SP[j * kRsThreads + tid] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+      sigma_p = sigma;
+      prev_p = p;
+    } else {
+#pragma unroll
+      for (int j = 0; j < V4; ++j) {
+        const float4 f = SP[j * kRsThreads + tid];
+        S[4 * j] = f.x;
+        S[4 * j + 1] = f.y;
+        S[4 * j + 2] = f.z;
+        S[4 * j + 3] = f.w;
+      }
+      sigma = sigma_p;
     }
+    // the beam's own token
+    load_slice<TIn, EL>(kc, a.k, in, e0, DK);
+    vc = row_ok ? to_f32(static_cast<const TIn*>(a.v)[in * size_t(a.d_v) + row]) : 0.f;
+    ac = expf(__ldg(a.g + in));
+    bc = __ldg(a.beta + in);
+    rs_transition<EL, LPR>(S, sigma, kc, vc, ac, bc);
     // o_t[i] = S_i . q_t
     load_slice<TIn, EL>(kc, a.q, in, e0, DK);
     float o = 0.f;
@@ -225,9 +282,15 @@ replayssm_kernel(StepArgs a) {
 template <typename TIn, int DK>
 static cudaError_t launch_rs_dk(const StepArgs& a, cudaStream_t stream) {
   using Sh = RsShape<DK>;
-  static_assert(rs_smem_bytes<DK>() <= 48 * 1024, "within the default shared-memory limit");
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = once_per_device(configured, [] {
+    return cudaFuncSetAttribute(replayssm_kernel<TIn, DK>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(rs_smem_bytes<DK>(4096)));
+  });
+  if (e != cudaSuccess) return e;
   const dim3 grid(unsigned(a.R) * a.H, unsigned((a.d_v + Sh::ROWS - 1) / Sh::ROWS));
-  replayssm_kernel<TIn, DK><<<grid, kRsThreads, rs_smem_bytes<DK>(), stream>>>(a);
+  replayssm_kernel<TIn, DK><<<grid, kRsThreads, rs_smem_bytes<DK>(a.B), stream>>>(a);
   return cudaGetLastError();
 }
 
