@@ -21,8 +21,10 @@
  * over the records of the beam's chain ("Scientific Impact Assessment: OneLA", §1: append-only
  * records of O(d_v + d_k) per beam, projection replay through the key and query
  * contractions, one kernel reusing S_ctx across beams; the OneLA listing's Abstract: records
- * are never moved or copied when beams are updated). The FullState path keeps one d_v x d_k
- * state per beam (the practice the Abstract contrasts with) and is kept as a comparison.
+ * are never moved or copied when beams are updated). Two comparison paths implement the
+ * practices the Abstract contrasts with: FullState keeps one d_v x d_k state per beam, and the
+ * history-replay path (REPLAYSSM) keeps no state at all and rebuilds every beam's state from
+ * S_ctx over its chain's raw tokens at every step.
  *
  * Conventions (every entry point)
  * -------------------------------
