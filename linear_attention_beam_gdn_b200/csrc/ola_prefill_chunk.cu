@@ -4,29 +4,38 @@
 // from one recurrent state derived from the shared prompt. Token by token (alpha = exp(g)):
 //     w_p = beta_p (v_p - alpha_p S k_p),    S <- alpha_p S + w_p k_p^T.
 // The pages give only this token recurrence; the chunked form below is derived from it. For a
-// chunk of C tokens j = 1..C entered with state S0, let G_j = g_1 + ... + g_j (inclusive) and
-// a_j = exp(G_j). Unrolling the recurrence inside the chunk gives, for every token j,
-//     w_j + sum_{m<j} L_jm w_m = R_j := beta_j (v_j - a_j S0 k_j),
-//     L_jm = beta_j e^{G_j - G_m} (k_j . k_m)                              (m < j),
-//     S_C  = a_C S0 + sum_j e^{G_C - G_j} w_j k_j^T.
-// With T = (I + L)^-1 (unit lower triangular, a function of the chunk's keys and gates only):
-//     Z = S0 K^T,   R = beta (V - a Z),   W = R T^T,   S_C = a_C S0 + (W D) K,
-// D = diag(e^{G_C - G_j}); rows of S are independent (row i only meets v[i]). Every exponent
-// is a difference G_j - G_m <= 0 or G <= 0, so no factor exceeds 1.
+// chunk of C tokens j = 1..C entered with state S0, let G_j = g_1 + ... + g_j (inclusive),
+// a_j = exp(G_j) and D_j = exp(G_C - G_j). Unrolling the recurrence inside the chunk gives
+//     w_j + sum_{m<j} beta_j e^{G_j - G_m} (k_j . k_m) w_m = beta_j (v_j - a_j S0 k_j),
+//     S_C = a_C S0 + sum_j D_j w_j k_j^T.
+// The decay factors of the triangular system are a diagonal similarity, E A E^-1 with
+// E = diag(e^{G_j}) and A = I + diag(beta) K~ (K~ the strictly lower part of K K^T), so with
+// T = A^-1 (unit lower triangular, no exponentials) w_m = sum_j e^{G_m - G_j} T_mj (...)_j.
+// Collecting the chunk's decayed writes Y = [D_m w_m]_m (d_v x C), every exponential becomes a
+// per-token scalar:
+//     Y = U + S0 N,   U = V^T M1,   N = K^T M2,
+//     M1_jm = beta_j D_j T_mj,   M2_jm = -a_C beta_j T_mj,
+// so the state meets the chunk in one product, and S_C = a_C S0 + Y K. U and N depend only on
+// the chunk's inputs and are formed off the state chain; no exponent is positive.
 //
-// One CTA per (request, head), one per SM (tensor memory: 384 of 512 columns):
-//   warps 0-3, 10-13  two precompute groups taking alternate chunks, ahead of the state
-//              chain: gates (prefix sums, a, D), K K^T on warp-level MMA from the key tile
-//              (exact bf16 products), L, T in fp32 by 16 x 16 blocks (diagonal blocks by
-//              forward substitution, then T_ba = -T_bb sum_{a <= c < b} L_bc T_ca by block
-//              distance), T as bf16 hi + lo tiles
-//   warps 4-7  state rows (thread = row = tensor-memory lane): R, W D, and the state entering
-//              the next chunk (its bf16 hi + lo for Z, and a_C S for the accumulation)
+// One CTA per (request, head), one per SM (tensor memory: all 512 columns):
+//   warp 14    tcgen05.mma off the chain: the Gram matrix K K^T of each chunk (exact bf16
+//              products) once its key tile has landed, and N once the chunk's M2 tiles are
+//              written
+//   warps 0-3, 10-13  two precompute groups taking alternate chunks, ahead of the state chain:
+//              gates (prefix sums, beta D, -a_C beta), L = diag(beta) K~ from the Gram matrix,
+//              T = (I + L)^-1 in fp32 by 16 x 16 blocks (diagonal blocks by forward
+//              substitution, the others by block products over two halves of 32),
+//              M1 and M2 as bf16 hi + lo tiles
+//   warp 9     tcgen05.mma, the chain: P = U + S N (S hi + lo in tensor memory), S += Y K
+//              (keys as MN-major B), then U of the next chunk into P's columns
+//   warps 4-7  state rows (thread = row = tensor-memory lane): Y = P as bf16 hi + lo, the
+//              state leaving the chunk (its bf16 hi + lo for P, and a_C S for the accumulation),
+//              and, while S is updated, the next chunk's N as bf16 hi + lo tiles
 //   warp 8     TMA: key and value tiles of each chunk, three stages
-//   warp 9     tcgen05.mma: Z = S K^T (S hi + lo in tensor memory),
-//              W = R T^T (three products of hi/lo parts), S += (W D) K (keys as MN-major B)
-// fp32 values enter the tensor cores as hi = bf16(x) plus lo = bf16(x - hi) (about 16
-// significant bits); the lo x lo product is dropped; keys are bf16 already and exact.
+// Per chunk the chain is P, the Y split, S += Y K and the state's split. fp32 values enter the
+// tensor cores as hi = bf16(x) plus lo = bf16(x - hi) (about 16 significant bits); the lo x lo
+// product is dropped; keys and values are bf16 already and exact.
 #include "ola_device.cuh"
 
 namespace ola {
@@ -36,49 +45,58 @@ namespace {
 constexpr int kC = 64;             // tokens per chunk
 constexpr int kD = 128;            // d_k = d_v
 constexpr int kStages = 3;
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr int kWRow = 4;           // first state-row warp
 constexpr int kWTma = 8;
 constexpr int kWMma = 9;
 constexpr int kWPre1 = 10;         // first warp of the second precompute group
+constexpr int kWGram = 14;
 constexpr int kBarPre = 1;         // named barriers 1 and 2: the two precompute groups
 
-// tensor memory columns (lane = state row)
-constexpr uint32_t kTS = 0;        // S fp32, 128 columns
+// tensor memory columns
+constexpr uint32_t kTS = 0;        // S fp32, 128 columns (lane = state row)
 constexpr uint32_t kTSH = 128;     // S as bf16 hi, two per column (64 columns)
 constexpr uint32_t kTSL = 192;     // S as bf16 lo
-constexpr uint32_t kTZ = 256;      // Z, then W: fp32, one column per token (64)
-constexpr uint32_t kTRH = 320;     // R, then W D: bf16 hi (32 columns)
-constexpr uint32_t kTRL = 352;     // ... bf16 lo
+constexpr uint32_t kTP = 256;      // P = U + S N = Y: fp32, one column per token (64)
+constexpr uint32_t kTYH = 320;     // Y as bf16 hi (32 columns)
+constexpr uint32_t kTYL = 352;     // ... bf16 lo
+constexpr uint32_t kTN = 384;      // N fp32 (lane = key column, one column per token)
+constexpr uint32_t kTG = 448;      // K K^T fp32 (lanes 0-63 = token)
 
 // shared memory, offsets from a 1024-byte aligned base
 constexpr uint32_t kTile = kC * kD * 2;                        // 16 KB: [2 col blocks][64][128 B]
-constexpr uint32_t kTTile = kC * kC * 2;                       // 8 KB: [64][64] bf16, sw128
-constexpr int kScFloats = 3 * kC + 4;                          // a, beta, D, a_C (+ pad)
+constexpr uint32_t kMTile = kC * kC * 2;                       // 8 KB: [64][64] bf16, sw128
+constexpr uint32_t kNTile = kD * kC * 2;                       // 16 KB: [128 key columns][64]
+constexpr int kScFloats = 3 * kC + 4;                          // beta, beta D, -a_C beta, a_C
 constexpr int kLd = kC + 1;                                    // padded fp32 row of L
 constexpr int kLdT = kC + 4;                                   // fp32 row of T (16-byte rows)
 constexpr uint32_t kOffK = 0;                                  // keys, 128-byte swizzle
-constexpr uint32_t kOffV = kOffK + kStages * kTile;            // values, no swizzle
-constexpr uint32_t kOffT = kOffV + kStages * kTile;            // T hi, T lo per stage
-constexpr uint32_t kOffSc = kOffT + kStages * 2 * kTTile;      // gate scalars per stage
-constexpr uint32_t kOffGrp = kOffSc + kStages * kScFloats * 4; // per precompute group:
-constexpr uint32_t kGL = 0;                                    //   L fp32 [64][65]
-constexpr uint32_t kGTf = kGL + kC * kLd * 4;                  //   T fp32 [64][68]
-constexpr uint32_t kGQ = kGTf + kC * kLdT * 4;                 //   block products [3][16][16]
-constexpr uint32_t kGG = kGQ + 3 * 256 * 4;                    //   G_j [64] + a warp total
-constexpr uint32_t kGrpBytes = kGG + (kC + 4) * 4;
+constexpr uint32_t kOffV = kOffK + kStages * kTile;            // values, 128-byte swizzle
+constexpr uint32_t kOffN = kOffV + kStages * kTile;            // N hi, N lo (one chunk)
+constexpr uint32_t kOffSc = kOffN + 2 * kNTile;                // gate scalars per stage
+constexpr uint32_t kOffGrp = kOffSc + 3072;                    // per precompute group:
+constexpr uint32_t kGL = 0;                                    //   L fp32 [64][65], then M1 hi, lo
+constexpr uint32_t kGTf = 17408;                               //   T fp32 [64][68], then M2 hi, lo
+constexpr uint32_t kGQ = kGTf + kC * kLdT * 4;                 //   block products [4][16][16]
+constexpr uint32_t kGG = kGQ + 4 * 256 * 4;                    //   G_j [64] + a warp total
+constexpr uint32_t kGrpBytes = 39936;
 constexpr uint32_t kOffBar = kOffGrp + 2 * kGrpBytes;
-constexpr int kNumBars = 16;
+constexpr int kNumBars = 22;
 constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + holder, alignment
-static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
-static_assert((kOffGrp + kGTf) % 16 == 0 && (kOffGrp + kGQ) % 16 == 0 && kGrpBytes % 16 == 0,
+static_assert(kStages * kScFloats * 4 <= 3072, "gate scalars");
+static_assert(kC * kLd * 4 <= kGTf && 2 * kMTile <= kC * kLd * 4, "L region holds M1 hi + lo");
+static_assert(2 * kMTile <= kC * kLdT * 4, "T region holds M2 hi + lo");
+static_assert(kGG + (kC + 4) * 4 <= kGrpBytes && kGrpBytes % 1024 == 0, "group region");
+static_assert(kOffGrp % 1024 == 0 && kGTf % 1024 == 0 && kOffN % 1024 == 0 &&
+              kOffV % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert((kOffGrp + kGQ) % 16 == 0 && (kOffGrp + kGTf) % 16 == 0,
               "float4 rows of T and of the block products");
-static_assert(kOffT % 1024 == 0 && kOffV % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 struct ChunkArgs {
   CUtensorMap mk;     // k [R][P][H][128] bf16: box 64 x 1 x 64 x 1, 128-byte swizzle
-  CUtensorMap mv;     // v [R][P][H][128] bf16: same box, no swizzle
+  CUtensorMap mv;     // v [R][P][H][128] bf16: same box and swizzle
   const float* g;     // [R][P][H]
   const float* beta;  // [R][P][H]
   float* S;           // [R][H][128][128]
@@ -100,18 +118,21 @@ __device__ __forceinline__ bool bar_and(int id, int count, bool v) {
   return out != 0;
 }
 
+// hi = bf16(x), lo = bf16(x - hi) for a pair, packed two per word (the first in the low half).
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h2);
+  const __nv_bfloat162 l2 = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h2);
+  lo = *reinterpret_cast<const uint32_t*>(&l2);
+}
+
 // x (32 fp32, token order) as bf16 hi and lo words, two per word, the lower token in the low half.
 __device__ __forceinline__ void split32(const float (&x)[32], uint4 (&hi)[4], uint4 (&lo)[4]) {
   uint32_t* hw = reinterpret_cast<uint32_t*>(hi);
   uint32_t* lw = reinterpret_cast<uint32_t*>(lo);
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
-    const float2 hf = __bfloat1622float2(h2);
-    const __nv_bfloat162 l2 = __floats2bfloat162_rn(x[2 * e] - hf.x, x[2 * e + 1] - hf.y);
-    hw[e] = *reinterpret_cast<const uint32_t*>(&h2);
-    lw[e] = *reinterpret_cast<const uint32_t*>(&l2);
-  }
+  for (int e = 0; e < 16; ++e) split2(x[2 * e], x[2 * e + 1], hw[e], lw[e]);
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t t, float (&x)[32]) {
@@ -146,15 +167,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sm = align_smem_1024(smem_raw);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kOffBar);
   uint64_t* full = bar;              // [3] key and value tiles landed (TMA bytes)
-  uint64_t* empty = bar + 3;         // [3] stage reusable: MMA commit + 4 state-row warps
-  uint64_t* pre = bar + 6;           // [3] T tiles and gate scalars written: 4 precompute warps
-  uint64_t* z_full = bar + 9;        // Z in tensor memory
-  uint64_t* r_full = bar + 10;       // R hi/lo written (4 state-row warps)
-  uint64_t* w_full = bar + 11;       // W in tensor memory
-  uint64_t* y_full = bar + 12;       // W D hi/lo written (4 state-row warps)
-  uint64_t* s_full = bar + 13;       // S updated
-  uint64_t* shl_full = bar + 14;     // S hi/lo and a_C S written (4 state-row warps)
-  uint64_t* mma_done = bar + 15;     // every MMA of the CTA completed
+  uint64_t* empty = bar + 3;         // [3] stage reusable: chain MMA commit + 4 state-row warps
+  uint64_t* pre = bar + 6;           // [3] M1, M2 tiles and gate scalars written (4 warps)
+  uint64_t* kk_full = bar + 9;       // [2] Gram matrix of the group's chunk in tensor memory
+  uint64_t* kk_free = bar + 11;      // Gram matrix read (2 warps)
+  uint64_t* n_full = bar + 12;       // N of the next chunk in tensor memory
+  uint64_t* m_free = bar + 13;       // [2] the group's M1, M2 tiles read (U and N commits)
+  uint64_t* n_ready = bar + 15;      // N hi/lo tiles written (4 state-row warps)
+  uint64_t* p_full = bar + 16;       // P in tensor memory
+  uint64_t* y_full = bar + 17;       // Y hi/lo written (4 state-row warps)
+  uint64_t* s_full = bar + 18;       // S updated
+  uint64_t* shl_full = bar + 19;     // S hi/lo written (4 state-row warps)
+  uint64_t* mma_done = bar + 20;     // every chain MMA completed
+  uint64_t* gram_done = bar + 21;    // every Gram MMA completed
   uint32_t* holder = reinterpret_cast<uint32_t*>(bar + kNumBars);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = blockIdx.x / a.H, h = blockIdx.x % a.H;
@@ -166,13 +191,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 5);
       mbar_init(&pre[s], 4);
     }
-    mbar_init(z_full, 1);
-    mbar_init(r_full, 4);
-    mbar_init(w_full, 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&kk_full[g], 1);
+      mbar_init(&m_free[g], 2);
+    }
+    mbar_init(n_full, 1);
+    mbar_init(n_ready, 4);
+    mbar_init(kk_free, 2);
+    mbar_init(p_full, 1);
     mbar_init(y_full, 4);
     mbar_init(s_full, 1);
     mbar_init(shl_full, 4);
     mbar_init(mma_done, 1);
+    mbar_init(gram_done, 1);
     fence_barrier_init();
   }
   if (warp == kWMma) tmem_alloc(holder, 512);
@@ -181,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *holder;
   const uint32_t kbase = smem_u32(sm + kOffK);
+  const uint32_t vbase = smem_u32(sm + kOffV);
 
   if (warp == kWTma) {
     // ---------------------------------------------------------------- TMA producer
@@ -208,40 +240,96 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
         mbar_wait_bounded(&full[c % kStages], (c / kStages) & 1);
     }
-  } else if (warp == kWMma) {
-    // ---------------------------------------------------------------- MMA issue
-    const uint32_t id_z = idesc_bf16_f32(128, kC);
-    const uint32_t id_s = idesc_bf16_f32(128, kD) | (1u << 16);     // B (the keys) MN-major
-    bool ok = true;
+  } else if (warp == kWGram) {
+    // ---------------------------------------------------------------- Gram matrix and N
+    // K K^T: M = 128 (rows 0-63 the chunk's tokens; rows 64-127 read whatever lies past the
+    // tile in shared memory and are never used), N = 64 tokens, K = d_k.
+    // N = K^T M2: A the key tile read MN-major (d_k along M), B the M2 tiles.
+    // Order: Gram of chunk c + 1, then N of chunk c, so that neither group waits on the other.
+    const uint32_t id_g = idesc_bf16_f32(128, kC);
+    const uint32_t id_n = idesc_bf16_f32_amn(128, kC);
+    auto gram = [&](int c1) -> bool {
+      const int s1 = c1 % kStages;
+      const bool ok1 = __all_sync(kFull, mbar_wait_bounded(&full[s1], (c1 / kStages) & 1) &&
+                                             (c1 == 0 || mbar_wait_bounded(kk_free, (c1 - 1) & 1)));
+      tc_fence_after();
+      if (!ok1) return false;
+      const uint32_t kb = kbase + s1 * kTile;
+#pragma unroll 1
+      for (int ks = 0; ks < kD / 16; ++ks) {
+        const uint64_t d = sw128_kmajor_desc(kb + (ks >> 2) * 8192 + (ks & 3) * 32);
+        umma_bf16_w(tmem + kTG, d, d, id_g, ks != 0 ? 1u : 0u);
+      }
+      umma_commit_w(&kk_full[c1 & 1]);
+      return true;
+    };
+    bool ok = gram(0);
     for (int c = 0; c < nch && ok; ++c) {
-      const int s = c % kStages, n = c / kStages;
+      if (c + 1 < nch && !(ok = gram(c + 1))) break;
+      // N of chunk c once its M2 tiles are written and the previous N has left tensor memory
+      ok = __all_sync(kFull, mbar_wait_bounded(&pre[c % kStages], (c / kStages) & 1) &&
+                                 (c == 0 || mbar_wait_bounded(n_ready, (c - 1) & 1)));
+      tc_fence_after();
+      if (!ok) break;
+      const uint32_t kb = kbase + (c % kStages) * kTile;
+      const uint32_t mh = smem_u32(sm + kOffGrp + (c & 1) * kGrpBytes + kGTf), ml = mh + kMTile;
+#pragma unroll 1
+      for (int ks = 0; ks < kC / 16; ++ks) {
+        const uint64_t ak = sw128_mnmajor_desc(kb + ks * 2048, 8192, 1024);
+        umma_bf16_w(tmem + kTN, ak, sw128_kmajor_desc(mh + ks * 32), id_n, ks != 0 ? 1u : 0u);
+        umma_bf16_w(tmem + kTN, ak, sw128_kmajor_desc(ml + ks * 32), id_n, 1u);
+      }
+      umma_commit_w(n_full);
+      umma_commit_w(&m_free[c & 1]);
+    }
+    if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 45, 0);
+    umma_commit_w(gram_done);
+    mbar_wait_bounded(gram_done, 0);
+    __syncwarp();
+  } else if (warp == kWMma) {
+    // ---------------------------------------------------------------- chain MMA issue
+    const uint32_t id_u = idesc_bf16_f32_amn(128, kC);              // U: A MN-major
+    const uint32_t id_p = idesc_bf16_f32(128, kC) | (1u << 16);     // P: B (N tiles) MN-major
+    const uint32_t id_s = idesc_bf16_f32(128, kD) | (1u << 16);     // S: B (the keys) MN-major
+    const uint32_t nh = smem_u32(sm + kOffN), nl = nh + kNTile;
+    // U = V^T M1 of chunk c1 into P's columns (A: the value tile read MN-major, d_v along M)
+    auto issue_u = [&](int c1) -> bool {
+      const int s1 = c1 % kStages;
+      const uint32_t par = uint32_t(c1 / kStages) & 1u;
+      const bool ok1 = __all_sync(kFull, mbar_wait_bounded(&pre[s1], par) &&
+                                             mbar_wait_bounded(&full[s1], par));
+      tc_fence_after();
+      if (!ok1) return false;
+      const uint32_t vb = vbase + s1 * kTile;
+      const uint32_t mh = smem_u32(sm + kOffGrp + (c1 & 1) * kGrpBytes + kGL), ml = mh + kMTile;
+#pragma unroll 1
+      for (int ks = 0; ks < kC / 16; ++ks) {
+        const uint64_t av = sw128_mnmajor_desc(vb + ks * 2048, 8192, 1024);
+        umma_bf16_w(tmem + kTP, av, sw128_kmajor_desc(mh + ks * 32), id_u, ks != 0 ? 1u : 0u);
+        umma_bf16_w(tmem + kTP, av, sw128_kmajor_desc(ml + ks * 32), id_u, 1u);
+      }
+      umma_commit_w(&m_free[c1 & 1]);
+      return true;
+    };
+    bool ok = issue_u(0);
+    for (int c = 0; c < nch && ok; ++c) {
+      const int s = c % kStages;
       const uint32_t kb = kbase + s * kTile;
-      // Z = S K^T: M = 128 state rows, N = 64 tokens, K = d_k; S as hi + lo from tensor memory
-      ok = __all_sync(kFull, mbar_wait_bounded(&full[s], n & 1) &&
+      // P += S N: M = 128 state rows, N = 64 tokens, K = d_k; S_hi N_hi + S_hi N_lo + S_lo N_hi
+      ok = __all_sync(kFull, mbar_wait_bounded(n_ready, c & 1) &&
                                  mbar_wait_bounded(shl_full, c & 1));
       tc_fence_after();
       if (!ok) break;
 #pragma unroll 1
       for (int ks = 0; ks < kD / 16; ++ks) {
-        const uint64_t b = sw128_kmajor_desc(kb + (ks >> 2) * 8192 + (ks & 3) * 32);
-        umma_bf16_ts_w(tmem + kTZ, tmem + kTSH + ks * 8, b, id_z, ks != 0);
-        umma_bf16_ts_w(tmem + kTZ, tmem + kTSL + ks * 8, b, id_z, 1u);
+        const uint64_t bh = sw128_mnmajor_desc(nh + ks * 2048, 0, 1024);
+        const uint64_t bl = sw128_mnmajor_desc(nl + ks * 2048, 0, 1024);
+        umma_bf16_ts_w(tmem + kTP, tmem + kTSH + ks * 8, bh, id_p, 1u);
+        umma_bf16_ts_w(tmem + kTP, tmem + kTSH + ks * 8, bl, id_p, 1u);
+        umma_bf16_ts_w(tmem + kTP, tmem + kTSL + ks * 8, bh, id_p, 1u);
       }
-      umma_commit_w(z_full);
-      // W = R T^T: M = 128, N = 64 tokens, K = 64 tokens; R_hi T_hi + R_hi T_lo + R_lo T_hi
-      ok = __all_sync(kFull, mbar_wait_bounded(&pre[s], n & 1) && mbar_wait_bounded(r_full, c & 1));
-      tc_fence_after();
-      if (!ok) break;
-      const uint32_t th = smem_u32(sm + kOffT + s * 2 * kTTile), tl = th + kTTile;
-#pragma unroll 1
-      for (int ks = 0; ks < kC / 16; ++ks) {
-        const uint64_t bh = sw128_kmajor_desc(th + ks * 32), bl = sw128_kmajor_desc(tl + ks * 32);
-        umma_bf16_ts_w(tmem + kTZ, tmem + kTRH + ks * 8, bh, id_z, ks != 0);
-        umma_bf16_ts_w(tmem + kTZ, tmem + kTRH + ks * 8, bl, id_z, 1u);
-        umma_bf16_ts_w(tmem + kTZ, tmem + kTRL + ks * 8, bh, id_z, 1u);
-      }
-      umma_commit_w(w_full);
-      // S += (W D) K: M = 128, N = d_k, K = 64 tokens; the key tile read as an MN-major B
+      umma_commit_w(p_full);
+      // S += Y K: M = 128, N = d_k, K = 64 tokens; the key tile read as an MN-major B
       // (128-byte rows of 64 key columns per token, column blocks 8 KB apart, 8 tokens per 1 KB)
       ok = __all_sync(kFull, mbar_wait_bounded(y_full, c & 1));
       tc_fence_after();
@@ -249,11 +337,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int ks = 0; ks < kC / 16; ++ks) {
         const uint64_t b = sw128_mnmajor_desc(kb + ks * 2048, 8192, 1024);
-        umma_bf16_ts_w(tmem + kTS, tmem + kTRH + ks * 8, b, id_s, 1u);
-        umma_bf16_ts_w(tmem + kTS, tmem + kTRL + ks * 8, b, id_s, 1u);
+        umma_bf16_ts_w(tmem + kTS, tmem + kTYH + ks * 8, b, id_s, 1u);
+        umma_bf16_ts_w(tmem + kTS, tmem + kTYL + ks * 8, b, id_s, 1u);
       }
       umma_commit_w(s_full);
       umma_commit_w(&empty[s]);
+      if (c + 1 < nch) ok = issue_u(c + 1);      // P's columns were read by the Y split (y_full)
     }
     if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 41, 0);
     // every MMA issued has completed before tensor memory is released
@@ -264,6 +353,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- state rows
     const int sp = warp & 3, i = 32 * sp + lane;
     const uint32_t tl = tmem + (uint32_t(32 * sp) << 16);
+    // N of a chunk, from tensor memory (lane = key column) to the MN-major hi/lo tiles of the
+    // chain's P product: row = key column, 64 tokens in 128 bytes, 128-byte swizzle. Done by
+    // these warps between their own steps; the previous P product has read the tiles.
+    auto convert_n = [&](int c1) -> bool {
+      if (!__all_sync(kFull, mbar_wait_bounded(n_full, c1 & 1))) return false;
+      tc_fence_after();
+      unsigned char* th = sm + kOffN + uint32_t(i) * 128u;
+      unsigned char* tlo = th + kNTile;
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {                 // tokens 32 hf .. 32 hf + 31
+        float x[32];
+        tmem_ld32(tl + kTN + 32 * hf, x);
+        uint4 hi[4], lo[4];
+        split32(x, hi, lo);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t off = uint32_t(((4 * hf + q) ^ (i & 7)) << 4);
+          *reinterpret_cast<uint4*>(th + off) = hi[q];
+          *reinterpret_cast<uint4*>(tlo + off) = lo[q];
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(n_ready);
+      return true;
+    };
     {
       float z[32];
 #pragma unroll
@@ -275,79 +391,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(shl_full);
-    bool ok = true;
-    for (int c = 0; c < nch; ++c) {
-      const int s = c % kStages, n = c / kStages;
-      const float* sc = reinterpret_cast<const float*>(sm + kOffSc + s * kScFloats * 4);
-      ok = mbar_wait_bounded(&full[s], n & 1) && mbar_wait_bounded(&pre[s], n & 1) &&
-           mbar_wait_bounded(z_full, c & 1);
+    bool ok = convert_n(0);
+    for (int c = 0; c < nch && ok; ++c) {
+      const int s = c % kStages;
+      ok = mbar_wait_bounded(p_full, c & 1);
       if (!__all_sync(kFull, ok)) break;
       tc_fence_after();
-      // R_j = beta_j (v_j[i] - a_j Z_j)
-      const __nv_bfloat16* vt =
-          reinterpret_cast<const __nv_bfloat16*>(sm + kOffV + s * kTile + (i >> 6) * 8192) +
-          (i & 63);
+      // Y = P as bf16 hi + lo
 #pragma unroll 1
       for (int q = 0; q < 2; ++q) {
         float x[32];
-        tmem_ld32(tl + kTZ + 32 * q, x);
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const int j = 32 * q + 4 * e4;
-          const float4 av = *reinterpret_cast<const float4*>(sc + j);
-          const float4 bv = *reinterpret_cast<const float4*>(sc + kC + j);
-          x[4 * e4] = bv.x * (__bfloat162float(vt[j * 64]) - av.x * x[4 * e4]);
-          x[4 * e4 + 1] = bv.y * (__bfloat162float(vt[(j + 1) * 64]) - av.y * x[4 * e4 + 1]);
-          x[4 * e4 + 2] = bv.z * (__bfloat162float(vt[(j + 2) * 64]) - av.z * x[4 * e4 + 2]);
-          x[4 * e4 + 3] = bv.w * (__bfloat162float(vt[(j + 3) * 64]) - av.w * x[4 * e4 + 3]);
-        }
+        tmem_ld32(tl + kTP + 32 * q, x);
         uint4 hi[4], lo[4];
         split32(x, hi, lo);
-        tmem_st16(tl + kTRH + 16 * q, hi);
-        tmem_st16(tl + kTRL + 16 * q, lo);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(r_full);
-      // W D
-      ok = mbar_wait_bounded(w_full, c & 1);
-      if (!__all_sync(kFull, ok)) break;
-      tc_fence_after();
-#pragma unroll 1
-      for (int q = 0; q < 2; ++q) {
-        float x[32];
-        tmem_ld32(tl + kTZ + 32 * q, x);
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 dv = *reinterpret_cast<const float4*>(sc + 2 * kC + 32 * q + 4 * e4);
-          x[4 * e4] *= dv.x;
-          x[4 * e4 + 1] *= dv.y;
-          x[4 * e4 + 2] *= dv.z;
-          x[4 * e4 + 3] *= dv.w;
-        }
-        uint4 hi[4], lo[4];
-        split32(x, hi, lo);
-        tmem_st16(tl + kTRH + 16 * q, hi);
-        tmem_st16(tl + kTRL + 16 * q, lo);
+        tmem_st16(tl + kTYH + 16 * q, hi);
+        tmem_st16(tl + kTYL + 16 * q, lo);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(y_full);
-        mbar_arrive(&empty[s]);                      // done with this stage's values and scalars
+        mbar_arrive(&empty[s]);                      // done with this stage's scalars
       }
-      // the state leaving the chunk: bf16 hi + lo for the next Z, a_C S for the next update
       const bool last = c + 1 == nch;
       const int s1 = (c + 1) % kStages;
+      // the next chunk's N while S is updated, when it is already there
+      bool converted = last;
+      if (!last && __all_sync(kFull, mbar_test(n_full, (c + 1) & 1))) {
+        if (!(ok = convert_n(c + 1))) break;
+        converted = true;
+      }
+      // the state leaving the chunk, in one pass: bf16 hi + lo for the next P, then a_C S for
+      // the next accumulation
       ok = mbar_wait_bounded(s_full, c & 1);
       if (!last) ok = ok && mbar_wait_bounded(&pre[s1], ((c + 1) / kStages) & 1);
       if (!__all_sync(kFull, ok)) break;
       tc_fence_after();
       if (!last) {
-        // hi + lo for the next Z first (the chain waits on them), then a_C S for the next
-        // accumulation, which overlaps the next Z
+        const float aC =
+            reinterpret_cast<const float*>(sm + kOffSc + s1 * kScFloats * 4)[3 * kC];
 #pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           float x[32];
@@ -356,22 +439,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           split32(x, hi, lo);
           tmem_st16(tl + kTSH + 16 * q, hi);
           tmem_st16(tl + kTSL + 16 * q, lo);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(shl_full);
-        const float aC =
-            reinterpret_cast<const float*>(sm + kOffSc + s1 * kScFloats * 4)[3 * kC];
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          float x[32];
-          tmem_ld32(tl + kTS + 32 * q, x);
 #pragma unroll
           for (int e = 0; e < 32; ++e) x[e] *= aC;
           tmem_st32(tl + kTS + 32 * q, x);
         }
         tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(shl_full);
+        if (!converted && !(ok = convert_n(c + 1))) break;
       } else {
         float* dst = a.S + ((size_t(r) * a.H + h) * kD + i) * size_t(kD);
 #pragma unroll 1
@@ -388,9 +464,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 42, 0);
   } else {
     // ---------------------------------------------------------------- per-chunk precompute
-    // group grp takes chunks grp, grp + 2, ...; ptid = thread, pw = warp within the group
+    // group grp takes chunks grp, grp + 2, ...; ptid = thread within the group, qd = the
+    // warp's tensor-memory lane quarter
     const int grp = warp >= kWPre1 ? 1 : 0;
-    const int ptid = tid - 32 * (grp ? kWPre1 : 0), pw = ptid >> 5, pbar = kBarPre + grp;
+    const int ptid = tid - 32 * (grp ? kWPre1 : 0), pbar = kBarPre + grp;
+    const int qd = warp & 3;
     unsigned char* gb = sm + kOffGrp + grp * kGrpBytes;
     float* Lm = reinterpret_cast<float*>(gb + kGL);
     float* Tf = reinterpret_cast<float*>(gb + kGTf);
@@ -410,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float gj, bj;
     load_gates(grp, gj, bj);
     for (int c = grp; c < nch; c += 2) {
-      const int s = c % kStages, n = c / kStages;
+      const int s = c % kStages, n = c / kStages, cc = c >> 1;
       float* sc = reinterpret_cast<float*>(sm + kOffSc + s * kScFloats * 4);
       bool ok = n == 0 || mbar_wait_bounded(&empty[s], (n - 1) & 1);
       if (!bar_and(pbar, 128, ok)) {
@@ -431,75 +509,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ptid >= 32 && ptid < kC) G += Gs[kC];
       if (ptid < kC) Gs[ptid] = G;
       named_bar_sync(pbar, 128);
-      const float GC = Gs[kC - 1];
+      const float GC = Gs[kC - 1], aC = expf(GC);
       if (ptid < kC) {
-        sc[ptid] = expf(G);
-        sc[kC + ptid] = bcur;
-        sc[2 * kC + ptid] = expf(GC - G);
+        sc[ptid] = bcur;
+        sc[kC + ptid] = bcur * expf(GC - G);
+        sc[2 * kC + ptid] = -aC * bcur;
       }
-      if (ptid == 0) sc[3 * kC] = expf(GC);
-      // K K^T rows 16 w .. 16 w + 15 (group warp w) on warp-level MMA from the swizzled key
-      // tile, the 16-column tiles up to the diagonal only, and L from it (entries on or above
-      // the diagonal are never read)
-      ok = mbar_wait_bounded(&full[s], n & 1);
+      if (ptid == 0) sc[3 * kC] = aC;
+      named_bar_sync(pbar, 128);
+      // L = diag(beta) K~ from the Gram matrix in tensor memory, by the group's two warps on
+      // lane quarters 0 and 1 (thread = token j; entries on or above the diagonal are never
+      // read). L shares its shared memory with M1 and T with M2: the U and N products of the
+      // group's previous chunk have read them (m_free) before L is written.
+      if (qd < 2) {
+        ok = mbar_wait_bounded(&kk_full[grp], cc & 1) &&
+             (cc == 0 || mbar_wait_bounded(&m_free[grp], (cc - 1) & 1));
+        if (__all_sync(kFull, ok)) {
+          tc_fence_after();
+          const int j = 32 * qd + lane;
+          float x0[32], x1[32];
+          tmem_ld32(tmem + (uint32_t(32 * qd) << 16) + kTG, x0);
+          tmem_ld32(tmem + (uint32_t(32 * qd) << 16) + kTG + 32, x1);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(kk_free);
+          const float bjv = sc[j];
+          float* lrow = Lm + j * kLd;
+#pragma unroll
+          for (int m = 0; m < 32; ++m) {
+            lrow[m] = m < j ? bjv * x0[m] : 0.f;
+            lrow[32 + m] = 32 + m < j ? bjv * x1[m] : 0.f;
+          }
+        } else {
+          ok = false;
+        }
+      }
       if (!bar_and(pbar, 128, ok)) {
         if (ptid == 0) report_error(a.err, OLA_ERR_TIMEOUT, 44, c);
         break;
       }
-      {
-        const uint32_t kt = smem_u32(sm + kOffK + s * kTile);
-        // byte of the 8 keys columns x .. x + 7 of token t in the tile
-        auto kaddr = [&](int t, int x) {
-          return kt + uint32_t(x >> 6) * 8192u + uint32_t(t) * 128u +
-                 uint32_t((((x & 63) >> 3) ^ (t & 7)) << 4);
-        };
-        const int jb = pw;
-        uint32_t af[8][4];
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          ldsm_x4(kaddr(16 * jb + (lane & 15), 16 * ks + (lane >> 4) * 8), af[ks][0], af[ks][1],
-                  af[ks][2], af[ks][3]);
-        const int j0 = 16 * jb + (lane >> 2), j1 = j0 + 8, cq = 2 * (lane & 3);
-        const float G0 = Gs[j0], G1 = Gs[j1], b0 = sc[kC + j0], b1 = sc[kC + j1];
-        const int bt = ((lane >> 3) >> 1) * 8 + (lane & 7), bx = ((lane >> 3) & 1) * 8;
-        // the column tiles of the row block accumulate side by side: 2 (jb + 1) independent
-        // MMA chains of 8 steps instead of one long chain
-        float d[4][2][4];
-#pragma unroll
-        for (int mp = 0; mp < 4; ++mp)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) d[mp][0][e] = d[mp][1][e] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-          for (int mp = 0; mp < 4; ++mp) {
-            if (mp <= jb) {                              // warp-uniform
-              uint32_t b00, b01, b10, b11;
-              ldsm_x4(kaddr(16 * mp + bt, 16 * ks + bx), b00, b01, b10, b11);
-              mma_16816_bf16(d[mp][0], af[ks][0], af[ks][1], af[ks][2], af[ks][3], b00, b01);
-              mma_16816_bf16(d[mp][1], af[ks][0], af[ks][1], af[ks][2], af[ks][3], b10, b11);
-            }
-          }
-        }
-#pragma unroll
-        for (int mp = 0; mp < 4; ++mp) {
-          if (mp > jb) break;
-          const float* d0 = d[mp][0];
-          const float* d1 = d[mp][1];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int m = 16 * mp + cq + e, m8 = m + 8;
-            const float Gm = Gs[m], Gm8 = Gs[m8];
-            Lm[j0 * kLd + m] = m < j0 ? b0 * __expf(G0 - Gm) * d0[e] : 0.f;
-            Lm[j1 * kLd + m] = m < j1 ? b1 * __expf(G1 - Gm) * d0[2 + e] : 0.f;
-            Lm[j0 * kLd + m8] = m8 < j0 ? b0 * __expf(G0 - Gm8) * d1[e] : 0.f;
-            Lm[j1 * kLd + m8] = m8 < j1 ? b1 * __expf(G1 - Gm8) * d1[2 + e] : 0.f;
-          }
-        }
-      }
-      named_bar_sync(pbar, 128);
       // T = (I + L)^-1: the four 16 x 16 diagonal blocks by forward substitution (thread =
-      // column), then T_ba = -T_bb sum_{a <= c < b} L_bc T_ca by block distance b - a
+      // column), then the blocks below them
       if (ptid < kC) {
         const int o = 16 * (ptid >> 4), m = ptid & 15;
         // right-looking: once x[ii] is final it updates every later row (a chain of 15 steps)
@@ -515,71 +565,140 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int jj = 0; jj < 16; ++jj) Tf[(o + jj) * kLdT + o + m] = x[jj];
       }
       named_bar_sync(pbar, 128);
-      // task = (block pair, row y, 4 columns x0..x0+3)
-#pragma unroll 1
-      for (int dl = 1; dl < 4; ++dl) {
-        const int ntask = (4 - dl) * 64;
-        for (int o = ptid; o < ntask; o += 128) {
-          const int ab = o >> 6, bb = ab + dl, y = (o >> 2) & 15, x0 = (o & 3) * 4;
-          const float* lrow = Lm + (16 * bb + y) * kLd;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-          for (int cb = ab; cb < bb; ++cb) {
-#pragma unroll
-            for (int z = 0; z < 16; ++z) {
-              const float l = lrow[16 * cb + z];
-              const float4 t =
-                  *reinterpret_cast<const float4*>(Tf + (16 * cb + z) * kLdT + 16 * ab + x0);
-              acc.x += l * t.x;
-              acc.y += l * t.y;
-              acc.z += l * t.z;
-              acc.w += l * t.w;
-            }
-          }
-          *reinterpret_cast<float4*>(Qb + (ab * 16 + y) * 16 + x0) = acc;
+      // The off-diagonal blocks as two halves of 32: T = [[A, 0], [C, B]] with A, B the inverses
+      // of the two diagonal 32 x 32 parts and C = -B L_(23)(01) A. Each half's lower block
+      // first (T_10 = -T_11 L_10 T_00, T_32 = -T_33 L_32 T_22), then X = L_(23)(01) A and
+      // C = -B X; 16 x 16 block products, four barriers. Scratch (Qb): Y, then X.
+      {
+        // Y_h = L_(h+1)(h) T_hh for h = 0, 2 (thread = half, row y, 4 columns)
+        const int hb = 2 * (ptid >> 6), y = (ptid >> 2) & 15, x0 = (ptid & 3) * 4;
+        const float* lrow = Lm + (16 * hb + 16 + y) * kLd + 16 * hb;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int z = 0; z < 16; ++z) {
+          const float l = lrow[z];
+          const float4 t = *reinterpret_cast<const float4*>(Tf + (16 * hb + z) * kLdT + 16 * hb + x0);
+          acc.x += l * t.x;
+          acc.y += l * t.y;
+          acc.z += l * t.z;
+          acc.w += l * t.w;
         }
+        *reinterpret_cast<float4*>(Qb + (hb / 2) * 256 + y * 16 + x0) = acc;
         named_bar_sync(pbar, 128);
-        for (int o = ptid; o < ntask; o += 128) {
-          const int ab = o >> 6, bb = ab + dl, y = (o >> 2) & 15, x0 = (o & 3) * 4;
-          // T_bb row y (zeros past the diagonal)
-          const float* trow = Tf + (16 * bb + y) * kLdT + 16 * bb;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int z = 0; z < 16; ++z) {
-            const float tz = trow[z];
-            const float4 q = *reinterpret_cast<const float4*>(Qb + (ab * 16 + z) * 16 + x0);
-            acc.x -= tz * q.x;
-            acc.y -= tz * q.y;
-            acc.z -= tz * q.z;
-            acc.w -= tz * q.w;
-          }
-          *reinterpret_cast<float4*>(Tf + (16 * bb + y) * kLdT + 16 * ab + x0) = acc;
+        // T_(h+1)(h) = -T_(h+1)(h+1) Y_h
+        const float* trow = Tf + (16 * hb + 16 + y) * kLdT + 16 * hb + 16;
+        float4 t2 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int z = 0; z < 16; ++z) {
+          const float tz = trow[z];
+          const float4 q = *reinterpret_cast<const float4*>(Qb + (hb / 2) * 256 + z * 16 + x0);
+          t2.x -= tz * q.x;
+          t2.y -= tz * q.y;
+          t2.z -= tz * q.z;
+          t2.w -= tz * q.w;
         }
+        *reinterpret_cast<float4*>(Tf + (16 * hb + 16 + y) * kLdT + 16 * hb + x0) = t2;
         named_bar_sync(pbar, 128);
       }
-      // T as bf16 hi and lo, K-major tiles with the 128-byte swizzle: thread = half a row
+      {
+        // X_(br)(bc) = sum_{kb = bc..1} L_(br)(kb) T_(kb)(bc), br in {2, 3}, bc in {0, 1}
+        // (thread = block, rows 2 rp and 2 rp + 1, 4 columns); then C = -B X
+        const int blk = ptid >> 5, br = 2 + (blk >> 1), bc = blk & 1;
+        const int rp = (ptid >> 2) & 7, x0 = (ptid & 3) * 4;
+        const float* l0 = Lm + (16 * br + 2 * rp) * kLd;
+        const float* l1 = l0 + kLd;
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+#pragma unroll 1
+        for (int kb = bc; kb < 2; ++kb) {
+#pragma unroll 4
+          for (int z = 0; z < 16; ++z) {
+            const float u0 = l0[16 * kb + z], u1 = l1[16 * kb + z];
+            const float4 t =
+                *reinterpret_cast<const float4*>(Tf + (16 * kb + z) * kLdT + 16 * bc + x0);
+            a0.x += u0 * t.x;
+            a0.y += u0 * t.y;
+            a0.z += u0 * t.z;
+            a0.w += u0 * t.w;
+            a1.x += u1 * t.x;
+            a1.y += u1 * t.y;
+            a1.z += u1 * t.z;
+            a1.w += u1 * t.w;
+          }
+        }
+        float* xb = Qb + blk * 256;                     // X_(br)(bc) at ((br - 2) * 2 + bc)
+        *reinterpret_cast<float4*>(xb + (2 * rp) * 16 + x0) = a0;
+        *reinterpret_cast<float4*>(xb + (2 * rp + 1) * 16 + x0) = a1;
+        named_bar_sync(pbar, 128);
+        // C_(br)(bc) = -sum_{kb = 2..br} T_(br)(kb) X_(kb)(bc)
+        const float* t0 = Tf + (16 * br + 2 * rp) * kLdT;
+        const float* t1 = t0 + kLdT;
+        float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
+#pragma unroll 1
+        for (int kb = 2; kb <= br; ++kb) {
+          const float* xk = Qb + ((kb - 2) * 2 + bc) * 256;
+#pragma unroll 4
+          for (int z = 0; z < 16; ++z) {
+            const float u0 = t0[16 * kb + z], u1 = t1[16 * kb + z];
+            const float4 q = *reinterpret_cast<const float4*>(xk + z * 16 + x0);
+            c0.x -= u0 * q.x;
+            c0.y -= u0 * q.y;
+            c0.z -= u0 * q.z;
+            c0.w -= u0 * q.w;
+            c1.x -= u1 * q.x;
+            c1.y -= u1 * q.y;
+            c1.z -= u1 * q.z;
+            c1.w -= u1 * q.w;
+          }
+        }
+        *reinterpret_cast<float4*>(Tf + (16 * br + 2 * rp) * kLdT + 16 * bc + x0) = c0;
+        *reinterpret_cast<float4*>(Tf + (16 * br + 2 * rp + 1) * kLdT + 16 * bc + x0) = c1;
+        named_bar_sync(pbar, 128);
+      }
+      // M1 (over L) and M2 (over T) as bf16 hi and lo, K-major tiles with the 128-byte swizzle:
+      // tile row = output token (the N index), column = source token j (the K index); thread =
+      // half a row. T is read whole before M2 overwrites it.
       {
         const int jr = ptid >> 1, hf = ptid & 1;
-        unsigned char* thi = sm + kOffT + s * 2 * kTTile;
-        unsigned char* tlo = thi + kTTile;
+        float tv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int m0 = 32 * hf + e;
+          tv[e] = m0 <= jr ? Tf[jr * kLdT + m0] : 0.f;
+        }
+        // the scalars are loaded before the first tile store (the compiler cannot tell them
+        // apart from the tiles, so a load after a store would wait for it)
+        float s2[32];                    // M2 entries; tv becomes the M1 entries
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 bd = *reinterpret_cast<const float4*>(sc + kC + 32 * hf + 4 * e4);
+          const float4 na = *reinterpret_cast<const float4*>(sc + 2 * kC + 32 * hf + 4 * e4);
+          s2[4 * e4] = na.x * tv[4 * e4];
+          s2[4 * e4 + 1] = na.y * tv[4 * e4 + 1];
+          s2[4 * e4 + 2] = na.z * tv[4 * e4 + 2];
+          s2[4 * e4 + 3] = na.w * tv[4 * e4 + 3];
+          tv[4 * e4] *= bd.x;
+          tv[4 * e4 + 1] *= bd.y;
+          tv[4 * e4 + 2] *= bd.z;
+          tv[4 * e4 + 3] *= bd.w;
+        }
+        named_bar_sync(pbar, 128);
+        unsigned char* m1h = gb + kGL;
+        unsigned char* m2h = gb + kGTf;
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
           const int q = 4 * hf + qq;
-          uint32_t hw[4], lw[4];
+          uint32_t h1[4], l1[4], h2[4], l2[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int m0 = 8 * q + 2 * e;
-            const float t0 = m0 <= jr ? Tf[jr * kLdT + m0] : 0.f;
-            const float t1 = m0 + 1 <= jr ? Tf[jr * kLdT + m0 + 1] : 0.f;
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(t0, t1);
-            const float2 hf2 = __bfloat1622float2(h2);
-            const __nv_bfloat162 l2 = __floats2bfloat162_rn(t0 - hf2.x, t1 - hf2.y);
-            hw[e] = *reinterpret_cast<const uint32_t*>(&h2);
-            lw[e] = *reinterpret_cast<const uint32_t*>(&l2);
+            const int ix = 8 * qq + 2 * e;
+            split2(tv[ix], tv[ix + 1], h1[e], l1[e]);
+            split2(s2[ix], s2[ix + 1], h2[e], l2[e]);
           }
           const uint32_t off = uint32_t(jr) * 128u + uint32_t((q ^ (jr & 7)) << 4);
-          *reinterpret_cast<uint4*>(thi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(tlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          *reinterpret_cast<uint4*>(m1h + off) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+          *reinterpret_cast<uint4*>(m1h + kMTile + off) = make_uint4(l1[0], l1[1], l1[2], l1[3]);
+          *reinterpret_cast<uint4*>(m2h + off) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+          *reinterpret_cast<uint4*>(m2h + kMTile + off) = make_uint4(l2[0], l2[1], l2[2], l2[3]);
         }
       }
       fence_proxy_async_smem();
@@ -618,8 +737,9 @@ EncodeFn prompt_encoder() {
 }
 
 // [R][P][H][128] bf16 as a 4-D map (column, head, token, request); a 64 x 1 x 64 x 1 box is
-// one 64-column block of 64 consecutive tokens of one (request, head). Tokens past P read 0.
-bool make_prompt_map(CUtensorMap* map, const void* base, int R, int P, int H, bool swizzle) {
+// one 64-column block of 64 consecutive tokens of one (request, head), stored with the 128-byte
+// swizzle (the tensor cores read it K-major and MN-major). Tokens past P read 0.
+bool make_prompt_map(CUtensorMap* map, const void* base, int R, int P, int H) {
   EncodeFn fn = prompt_encoder();
   if (!fn) return false;
   cuuint64_t dims[4] = {cuuint64_t(kD), cuuint64_t(H), cuuint64_t(P), cuuint64_t(R)};
@@ -629,7 +749,7 @@ bool make_prompt_map(CUtensorMap* map, const void* base, int R, int P, int H, bo
   cuuint32_t es[4] = {1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
             box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
@@ -646,7 +766,7 @@ cudaError_t launch_prefill_chunk(int R, int H, int P, const void* k, const void*
                                  const float* g, const float* beta, float* S_out, int* err,
                                  cudaStream_t stream) {
   ChunkArgs a;
-  if (!make_prompt_map(&a.mk, k, R, P, H, true) || !make_prompt_map(&a.mv, v, R, P, H, false))
+  if (!make_prompt_map(&a.mk, k, R, P, H) || !make_prompt_map(&a.mv, v, R, P, H))
     return cudaErrorInvalidValue;
   a.g = g;
   a.beta = beta;
