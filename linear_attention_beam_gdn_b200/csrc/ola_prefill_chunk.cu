@@ -14,14 +14,14 @@
 // Collecting the chunk's decayed writes Y = [D_m w_m]_m (d_v x C), every exponential becomes a
 // per-token scalar:
 //     Y = U + S0 N,   U = V^T M1,   N = K^T M2,
-//     M1_jm = beta_j D_j T_mj,   M2_jm = -a_C beta_j T_mj,
+//     M1_jm = beta_j D_j T_mj,   M2_jm = -a_C beta_j T_mj = -a_j M1_jm,
 // so the state meets the chunk in one product, and S_C = a_C S0 + Y K. U and N depend only on
 // the chunk's inputs and are formed off the state chain; no exponent is positive.
 //
 // One CTA per (request, head), one per SM (tensor memory: all 512 columns):
-//   warp 14    tcgen05.mma off the chain: the Gram matrix K K^T of each chunk (exact bf16
-//              products) once its key tile has landed, and N once the chunk's M2 tiles are
-//              written
+//   warp 14    tcgen05.mma: the Gram matrix K K^T of each chunk (exact bf16 products) once
+//              its key tile has landed
+//   warp 15    tcgen05.mma: N of each chunk once its M2 tiles are written
 //   warps 0-3, 10-13  two precompute groups taking alternate chunks, ahead of the state chain:
 //              gates (prefix sums, beta D, -a_C beta), L = diag(beta) K~ from the Gram matrix,
 //              T = (I + L)^-1 in fp32 by 16 x 16 blocks (diagonal blocks by forward
@@ -45,12 +45,13 @@ namespace {
 constexpr int kC = 64;             // tokens per chunk
 constexpr int kD = 128;            // d_k = d_v
 constexpr int kStages = 3;
-constexpr int kThreads = 480;
+constexpr int kThreads = 512;
 constexpr int kWRow = 4;           // first state-row warp
 constexpr int kWTma = 8;
 constexpr int kWMma = 9;
 constexpr int kWPre1 = 10;         // first warp of the second precompute group
 constexpr int kWGram = 14;
+constexpr int kWN = 15;
 constexpr int kBarPre = 1;         // named barriers 1 and 2: the two precompute groups
 
 // tensor memory columns
@@ -67,21 +68,21 @@ constexpr uint32_t kTG = 448;      // K K^T fp32 (lanes 0-63 = token)
 constexpr uint32_t kTile = kC * kD * 2;                        // 16 KB: [2 col blocks][64][128 B]
 constexpr uint32_t kMTile = kC * kC * 2;                       // 8 KB: [64][64] bf16, sw128
 constexpr uint32_t kNTile = kD * kC * 2;                       // 16 KB: [128 key columns][64]
-constexpr int kScFloats = 3 * kC + 4;                          // beta, beta D, -a_C beta, a_C
-constexpr int kLd = kC + 1;                                    // padded fp32 row of L
+constexpr int kScFloats = 3 * kC + 4;                          // beta, beta D, -a, a_C
+constexpr int kLd = kC + 4;                                    // fp32 row of L (16-byte rows)
 constexpr int kLdT = kC + 4;                                   // fp32 row of T (16-byte rows)
 constexpr uint32_t kOffK = 0;                                  // keys, 128-byte swizzle
 constexpr uint32_t kOffV = kOffK + kStages * kTile;            // values, 128-byte swizzle
 constexpr uint32_t kOffN = kOffV + kStages * kTile;            // N hi, N lo (one chunk)
 constexpr uint32_t kOffSc = kOffN + 2 * kNTile;                // gate scalars per stage
 constexpr uint32_t kOffGrp = kOffSc + 3072;                    // per precompute group:
-constexpr uint32_t kGL = 0;                                    //   L fp32 [64][65], then M1 hi, lo
+constexpr uint32_t kGL = 0;                                    //   L fp32 [64][68], then M1 hi, lo
 constexpr uint32_t kGTf = 17408;                               //   T fp32 [64][68], then M2 hi, lo
 constexpr uint32_t kGQ = kGTf + kC * kLdT * 4;                 //   block products [4][16][16]
 constexpr uint32_t kGG = kGQ + 4 * 256 * 4;                    //   G_j [64] + a warp total
 constexpr uint32_t kGrpBytes = 39936;
 constexpr uint32_t kOffBar = kOffGrp + 2 * kGrpBytes;
-constexpr int kNumBars = 22;
+constexpr int kNumBars = 23;
 constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + holder, alignment
 static_assert(kStages * kScFloats * 4 <= 3072, "gate scalars");
 static_assert(kC * kLd * 4 <= kGTf && 2 * kMTile <= kC * kLd * 4, "L region holds M1 hi + lo");
@@ -159,6 +160,35 @@ __device__ __forceinline__ void tmem_st32(uint32_t t, const float (&x)[32]) {
   tmem_st16(t + 16, b);
 }
 
+// N of chunk c (in tensor memory, lane = key column) to the MN-major hi/lo tiles of the chain's
+// P product: row = key column i, 64 tokens in 128 bytes, 128-byte swizzle. Called by the
+// state-row warps between their own steps (the previous P product has read the tiles); out of
+// line, so that its three call sites share one copy of the code.
+static __device__ __noinline__ bool convert_n(uint32_t tl, unsigned char* th, int i,
+                                              uint64_t* n_full, uint64_t* n_ready, int c) {
+  if (!__all_sync(kFull, mbar_wait_bounded(n_full, c & 1))) return false;
+  tc_fence_after();
+  unsigned char* tlo = th + kNTile;
+#pragma unroll 1
+  for (int hf = 0; hf < 2; ++hf) {                   // tokens 32 hf .. 32 hf + 31
+    float x[32];
+    tmem_ld32(tl + kTN + 32 * hf, x);
+    uint4 hi[4], lo[4];
+    split32(x, hi, lo);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t off = uint32_t(((4 * hf + q) ^ (i & 7)) << 4);
+      *reinterpret_cast<uint4*>(th + off) = hi[q];
+      *reinterpret_cast<uint4*>(tlo + off) = lo[q];
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(n_ready);
+  return true;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -180,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* shl_full = bar + 19;     // S hi/lo written (4 state-row warps)
   uint64_t* mma_done = bar + 20;     // every chain MMA completed
   uint64_t* gram_done = bar + 21;    // every Gram MMA completed
+  uint64_t* n_done = bar + 22;       // every N MMA completed
   uint32_t* holder = reinterpret_cast<uint32_t*>(bar + kNumBars);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = blockIdx.x / a.H, h = blockIdx.x % a.H;
@@ -204,6 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(shl_full, 4);
     mbar_init(mma_done, 1);
     mbar_init(gram_done, 1);
+    mbar_init(n_done, 1);
     fence_barrier_init();
   }
   if (warp == kWMma) tmem_alloc(holder, 512);
@@ -241,32 +273,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_bounded(&full[c % kStages], (c / kStages) & 1);
     }
   } else if (warp == kWGram) {
-    // ---------------------------------------------------------------- Gram matrix and N
+    // ---------------------------------------------------------------- Gram matrix
     // K K^T: M = 128 (rows 0-63 the chunk's tokens; rows 64-127 read whatever lies past the
-    // tile in shared memory and are never used), N = 64 tokens, K = d_k.
-    // N = K^T M2: A the key tile read MN-major (d_k along M), B the M2 tiles.
-    // Order: Gram of chunk c + 1, then N of chunk c, so that neither group waits on the other.
+    // tile in shared memory and are never used), N = 64 tokens, K = d_k
     const uint32_t id_g = idesc_bf16_f32(128, kC);
-    const uint32_t id_n = idesc_bf16_f32_amn(128, kC);
-    auto gram = [&](int c1) -> bool {
-      const int s1 = c1 % kStages;
-      const bool ok1 = __all_sync(kFull, mbar_wait_bounded(&full[s1], (c1 / kStages) & 1) &&
-                                             (c1 == 0 || mbar_wait_bounded(kk_free, (c1 - 1) & 1)));
+    bool ok = true;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int s = c % kStages;
+      ok = __all_sync(kFull, mbar_wait_bounded(&full[s], (c / kStages) & 1) &&
+                                 (c == 0 || mbar_wait_bounded(kk_free, (c - 1) & 1)));
       tc_fence_after();
-      if (!ok1) return false;
-      const uint32_t kb = kbase + s1 * kTile;
+      if (!ok) break;
+      const uint32_t kb = kbase + s * kTile;
 #pragma unroll 1
       for (int ks = 0; ks < kD / 16; ++ks) {
         const uint64_t d = sw128_kmajor_desc(kb + (ks >> 2) * 8192 + (ks & 3) * 32);
         umma_bf16_w(tmem + kTG, d, d, id_g, ks != 0 ? 1u : 0u);
       }
-      umma_commit_w(&kk_full[c1 & 1]);
-      return true;
-    };
-    bool ok = gram(0);
+      umma_commit_w(&kk_full[c & 1]);
+    }
+    if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 45, 0);
+    umma_commit_w(gram_done);
+    mbar_wait_bounded(gram_done, 0);
+    __syncwarp();
+  } else if (warp == kWN) {
+    // ---------------------------------------------------------------- N = K^T M2
+    // A the key tile read MN-major (d_k along M), B the chunk's M2 tiles; once they are written
+    // and the previous N has left tensor memory
+    const uint32_t id_n = idesc_bf16_f32_amn(128, kC);
+    bool ok = true;
     for (int c = 0; c < nch && ok; ++c) {
-      if (c + 1 < nch && !(ok = gram(c + 1))) break;
-      // N of chunk c once its M2 tiles are written and the previous N has left tensor memory
       ok = __all_sync(kFull, mbar_wait_bounded(&pre[c % kStages], (c / kStages) & 1) &&
                                  (c == 0 || mbar_wait_bounded(n_ready, (c - 1) & 1)));
       tc_fence_after();
@@ -282,9 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit_w(n_full);
       umma_commit_w(&m_free[c & 1]);
     }
-    if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 45, 0);
-    umma_commit_w(gram_done);
-    mbar_wait_bounded(gram_done, 0);
+    if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 47, 0);
+    umma_commit_w(n_done);
+    mbar_wait_bounded(n_done, 0);
     __syncwarp();
   } else if (warp == kWMma) {
     // ---------------------------------------------------------------- chain MMA issue
@@ -311,37 +347,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit_w(&m_free[c1 & 1]);
       return true;
     };
-    bool ok = issue_u(0);
-    for (int c = 0; c < nch && ok; ++c) {
-      const int s = c % kStages;
-      const uint32_t kb = kbase + s * kTile;
-      // P += S N: M = 128 state rows, N = 64 tokens, K = d_k; S_hi N_hi + S_hi N_lo + S_lo N_hi
-      ok = __all_sync(kFull, mbar_wait_bounded(n_ready, c & 1) &&
-                                 mbar_wait_bounded(shl_full, c & 1));
-      tc_fence_after();
-      if (!ok) break;
+    // step c: the chain of chunk c (c >= 0), then U of chunk c + 1 (one call site for U)
+    bool ok = true;
+    for (int c = -1; c < nch && ok; ++c) {
+      if (c >= 0) {
+        const int s = c % kStages;
+        const uint32_t kb = kbase + s * kTile;
+        // P += S N: M = 128 state rows, N = 64 tokens, K = d_k; S_hi N_hi + S_hi N_lo + S_lo N_hi
+        ok = __all_sync(kFull, mbar_wait_bounded(n_ready, c & 1) &&
+                                   mbar_wait_bounded(shl_full, c & 1));
+        tc_fence_after();
+        if (!ok) break;
 #pragma unroll 1
-      for (int ks = 0; ks < kD / 16; ++ks) {
-        const uint64_t bh = sw128_mnmajor_desc(nh + ks * 2048, 0, 1024);
-        const uint64_t bl = sw128_mnmajor_desc(nl + ks * 2048, 0, 1024);
-        umma_bf16_ts_w(tmem + kTP, tmem + kTSH + ks * 8, bh, id_p, 1u);
-        umma_bf16_ts_w(tmem + kTP, tmem + kTSH + ks * 8, bl, id_p, 1u);
-        umma_bf16_ts_w(tmem + kTP, tmem + kTSL + ks * 8, bh, id_p, 1u);
-      }
-      umma_commit_w(p_full);
-      // S += Y K: M = 128, N = d_k, K = 64 tokens; the key tile read as an MN-major B
-      // (128-byte rows of 64 key columns per token, column blocks 8 KB apart, 8 tokens per 1 KB)
-      ok = __all_sync(kFull, mbar_wait_bounded(y_full, c & 1));
-      tc_fence_after();
-      if (!ok) break;
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint64_t bh = sw128_mnmajor_desc(nh + ks * 2048, 0, 1024);
+          const uint64_t bl = sw128_mnmajor_desc(nl + ks * 2048, 0, 1024);
+          umma_bf16_ts_w(tmem + kTP, tmem + kTSH + ks * 8, bh, id_p, 1u);
+          umma_bf16_ts_w(tmem + kTP, tmem + kTSH + ks * 8, bl, id_p, 1u);
+          umma_bf16_ts_w(tmem + kTP, tmem + kTSL + ks * 8, bh, id_p, 1u);
+        }
+        umma_commit_w(p_full);
+        // S += Y K: M = 128, N = d_k, K = 64 tokens; the key tile read as an MN-major B
+        // (128-byte rows of 64 key columns per token, column blocks 8 KB apart, 8 tokens per 1 KB)
+        ok = __all_sync(kFull, mbar_wait_bounded(y_full, c & 1));
+        tc_fence_after();
+        if (!ok) break;
 #pragma unroll 1
-      for (int ks = 0; ks < kC / 16; ++ks) {
-        const uint64_t b = sw128_mnmajor_desc(kb + ks * 2048, 8192, 1024);
-        umma_bf16_ts_w(tmem + kTS, tmem + kTYH + ks * 8, b, id_s, 1u);
-        umma_bf16_ts_w(tmem + kTS, tmem + kTYL + ks * 8, b, id_s, 1u);
+        for (int ks = 0; ks < kC / 16; ++ks) {
+          const uint64_t b = sw128_mnmajor_desc(kb + ks * 2048, 8192, 1024);
+          umma_bf16_ts_w(tmem + kTS, tmem + kTYH + ks * 8, b, id_s, 1u);
+          umma_bf16_ts_w(tmem + kTS, tmem + kTYL + ks * 8, b, id_s, 1u);
+        }
+        umma_commit_w(s_full);
+        umma_commit_w(&empty[s]);
       }
-      umma_commit_w(s_full);
-      umma_commit_w(&empty[s]);
       if (c + 1 < nch) ok = issue_u(c + 1);      // P's columns were read by the Y split (y_full)
     }
     if (!ok && lane == 0) report_error(a.err, OLA_ERR_TIMEOUT, 41, 0);
@@ -353,33 +392,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- state rows
     const int sp = warp & 3, i = 32 * sp + lane;
     const uint32_t tl = tmem + (uint32_t(32 * sp) << 16);
-    // N of a chunk, from tensor memory (lane = key column) to the MN-major hi/lo tiles of the
-    // chain's P product: row = key column, 64 tokens in 128 bytes, 128-byte swizzle. Done by
-    // these warps between their own steps; the previous P product has read the tiles.
-    auto convert_n = [&](int c1) -> bool {
-      if (!__all_sync(kFull, mbar_wait_bounded(n_full, c1 & 1))) return false;
-      tc_fence_after();
-      unsigned char* th = sm + kOffN + uint32_t(i) * 128u;
-      unsigned char* tlo = th + kNTile;
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {                 // tokens 32 hf .. 32 hf + 31
-        float x[32];
-        tmem_ld32(tl + kTN + 32 * hf, x);
-        uint4 hi[4], lo[4];
-        split32(x, hi, lo);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t off = uint32_t(((4 * hf + q) ^ (i & 7)) << 4);
-          *reinterpret_cast<uint4*>(th + off) = hi[q];
-          *reinterpret_cast<uint4*>(tlo + off) = lo[q];
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(n_ready);
-      return true;
-    };
     {
       float z[32];
 #pragma unroll
@@ -391,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(shl_full);
-    bool ok = convert_n(0);
+    bool ok = convert_n(tl, sm + kOffN + uint32_t(i) * 128u, i, n_full, n_ready, 0);
     for (int c = 0; c < nch && ok; ++c) {
       const int s = c % kStages;
       ok = mbar_wait_bounded(p_full, c & 1);
@@ -419,7 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the next chunk's N while S is updated, when it is already there
       bool converted = last;
       if (!last && __all_sync(kFull, mbar_test(n_full, (c + 1) & 1))) {
-        if (!(ok = convert_n(c + 1))) break;
+        if (!(ok = convert_n(tl, sm + kOffN + uint32_t(i) * 128u, i, n_full, n_ready, c + 1)))
+          break;
         converted = true;
       }
       // the state leaving the chunk, in one pass: bf16 hi + lo for the next P, then a_C S for
@@ -447,7 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(shl_full);
-        if (!converted && !(ok = convert_n(c + 1))) break;
+        if (!converted &&
+            !(ok = convert_n(tl, sm + kOffN + uint32_t(i) * 128u, i, n_full, n_ready, c + 1)))
+          break;
       } else {
         float* dst = a.S + ((size_t(r) * a.H + h) * kD + i) * size_t(kD);
 #pragma unroll 1
@@ -513,13 +528,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ptid < kC) {
         sc[ptid] = bcur;
         sc[kC + ptid] = bcur * expf(GC - G);
-        sc[2 * kC + ptid] = -aC * bcur;
+        sc[2 * kC + ptid] = -expf(G);
       }
       if (ptid == 0) sc[3 * kC] = aC;
       named_bar_sync(pbar, 128);
       // L = diag(beta) K~ from the Gram matrix in tensor memory, by the group's two warps on
-      // lane quarters 0 and 1 (thread = token j; entries on or above the diagonal are never
-      // read). L shares its shared memory with M1 and T with M2: the U and N products of the
+      // lane quarters 0 and 1 (thread = token j; whole rows are written, but only the entries
+      // below the diagonal are ever read). L shares its shared memory with M1 and T with M2: the U and N products of the
       // group's previous chunk have read them (m_free) before L is written.
       if (qd < 2) {
         ok = mbar_wait_bounded(&kk_full[grp], cc & 1) &&
@@ -534,11 +549,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(kk_free);
           const float bjv = sc[j];
-          float* lrow = Lm + j * kLd;
+          float4* lrow = reinterpret_cast<float4*>(Lm + j * kLd);
 #pragma unroll
-          for (int m = 0; m < 32; ++m) {
-            lrow[m] = m < j ? bjv * x0[m] : 0.f;
-            lrow[32 + m] = 32 + m < j ? bjv * x1[m] : 0.f;
+          for (int m4 = 0; m4 < 8; ++m4) {
+            lrow[m4] = make_float4(bjv * x0[4 * m4], bjv * x0[4 * m4 + 1], bjv * x0[4 * m4 + 2],
+                                   bjv * x0[4 * m4 + 3]);
+            lrow[8 + m4] = make_float4(bjv * x1[4 * m4], bjv * x1[4 * m4 + 1],
+                                       bjv * x1[4 * m4 + 2], bjv * x1[4 * m4 + 3]);
           }
         } else {
           ok = false;
@@ -654,49 +671,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<float4*>(Tf + (16 * br + 2 * rp + 1) * kLdT + 16 * bc + x0) = c1;
         named_bar_sync(pbar, 128);
       }
-      // M1 (over L) and M2 (over T) as bf16 hi and lo, K-major tiles with the 128-byte swizzle:
-      // tile row = output token (the N index), column = source token j (the K index); thread =
-      // half a row. T is read whole before M2 overwrites it.
+      // M1 (over L), then M2 (over T) as bf16 hi and lo, K-major tiles with the 128-byte
+      // swizzle: tile row = output token (the N index), column = source token j (the K index);
+      // thread = half a row, 16 bytes (8 columns) at a time. M2_jm = M1_jm (-a_j), formed from
+      // M1's hi + lo once every T entry has been read.
       {
         const int jr = ptid >> 1, hf = ptid & 1;
-        float tv[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int m0 = 32 * hf + e;
-          tv[e] = m0 <= jr ? Tf[jr * kLdT + m0] : 0.f;
-        }
-        // the scalars are loaded before the first tile store (the compiler cannot tell them
-        // apart from the tiles, so a load after a store would wait for it)
-        float s2[32];                    // M2 entries; tv becomes the M1 entries
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 bd = *reinterpret_cast<const float4*>(sc + kC + 32 * hf + 4 * e4);
-          const float4 na = *reinterpret_cast<const float4*>(sc + 2 * kC + 32 * hf + 4 * e4);
-          s2[4 * e4] = na.x * tv[4 * e4];
-          s2[4 * e4 + 1] = na.y * tv[4 * e4 + 1];
-          s2[4 * e4 + 2] = na.z * tv[4 * e4 + 2];
-          s2[4 * e4 + 3] = na.w * tv[4 * e4 + 3];
-          tv[4 * e4] *= bd.x;
-          tv[4 * e4 + 1] *= bd.y;
-          tv[4 * e4 + 2] *= bd.z;
-          tv[4 * e4 + 3] *= bd.w;
-        }
-        named_bar_sync(pbar, 128);
         unsigned char* m1h = gb + kGL;
         unsigned char* m2h = gb + kGTf;
-#pragma unroll
+#pragma unroll 1
         for (int qq = 0; qq < 4; ++qq) {
-          const int q = 4 * hf + qq;
-          uint32_t h1[4], l1[4], h2[4], l2[4];
+          const int q = 4 * hf + qq, m0 = 8 * q;
+          const float4 t0 = *reinterpret_cast<const float4*>(Tf + jr * kLdT + m0);
+          const float4 t1 = *reinterpret_cast<const float4*>(Tf + jr * kLdT + m0 + 4);
+          const float4 b0 = *reinterpret_cast<const float4*>(sc + kC + m0);
+          const float4 b1 = *reinterpret_cast<const float4*>(sc + kC + m0 + 4);
+          // entries past the diagonal are not T's (zero, or stale in blocks above it)
+          const float t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+          const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            split2(m0 + 2 * e <= jr ? t[2 * e] * b[2 * e] : 0.f,
+                   m0 + 2 * e + 1 <= jr ? t[2 * e + 1] * b[2 * e + 1] : 0.f, hw[e], lw[e]);
+          const uint32_t off = uint32_t(jr) * 128u + uint32_t((q ^ (jr & 7)) << 4);
+          *reinterpret_cast<uint4*>(m1h + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(m1h + kMTile + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+        named_bar_sync(pbar, 128);
+#pragma unroll 1
+        for (int qq = 0; qq < 4; ++qq) {
+          const int q = 4 * hf + qq, m0 = 8 * q;
+          const uint32_t off = uint32_t(jr) * 128u + uint32_t((q ^ (jr & 7)) << 4);
+          const uint4 h = *reinterpret_cast<const uint4*>(m1h + off);
+          const uint4 l = *reinterpret_cast<const uint4*>(m1h + kMTile + off);
+          const float4 a0 = *reinterpret_cast<const float4*>(sc + 2 * kC + m0);
+          const float4 a1 = *reinterpret_cast<const float4*>(sc + 2 * kC + m0 + 4);
+          const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
+          const float na[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+          uint32_t h2[4], l2[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int ix = 8 * qq + 2 * e;
-            split2(tv[ix], tv[ix + 1], h1[e], l1[e]);
-            split2(s2[ix], s2[ix + 1], h2[e], l2[e]);
+            // bf16 pairs back to fp32: the low half holds the first column
+            const float x0 = __uint_as_float(hw[e] << 16) + __uint_as_float(lw[e] << 16);
+            const float x1 =
+                __uint_as_float(hw[e] & 0xffff0000u) + __uint_as_float(lw[e] & 0xffff0000u);
+            split2(x0 * na[2 * e], x1 * na[2 * e + 1], h2[e], l2[e]);
           }
-          const uint32_t off = uint32_t(jr) * 128u + uint32_t((q ^ (jr & 7)) << 4);
-          *reinterpret_cast<uint4*>(m1h + off) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
-          *reinterpret_cast<uint4*>(m1h + kMTile + off) = make_uint4(l1[0], l1[1], l1[2], l1[3]);
           *reinterpret_cast<uint4*>(m2h + off) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
           *reinterpret_cast<uint4*>(m2h + kMTile + off) = make_uint4(l2[0], l2[1], l2[2], l2[3]);
         }
