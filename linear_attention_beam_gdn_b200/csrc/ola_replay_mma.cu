@@ -559,7 +559,7 @@ replay_mma_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* _
     // Per unit, from the staged data only (nothing here waits for a tensor-core result, so the
     // warp runs ahead): the decay table, the per-position scalars and the append of alpha_p.
     for (int i = 0; i < n_my; ++i) {
-      const int sb = i % NB, ac = i % NA, db = i & 1;
+      const int sb = i % NB, db = i & 1;
       bool ok = mbar_wait_bounded(&fullB[sb], (i / NB) & 1);
       if (i >= 2) ok = ok && mbar_wait_bounded(&dec_free[db], ((i - 2) >> 1) & 1);      // DEC[db] free
       if (!__all_sync(kFull, ok)) {

@@ -304,8 +304,7 @@ replay_pipe_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* 
     const __nv_bfloat16* krec = kout;
     for (int i = 0; i < n_my; ++i) {
       const int u = ubeg + i, s = i % NS, n = i / NS;
-      const int rh = u / n_chunks, c0 = (u % n_chunks) * NB;
-      const int r = rh / a.H, h = rh % a.H;
+      const int rh = u / n_chunks;
       const bool new_s = rh != prev_rh;
       if (new_s) {
         ++sver;
@@ -422,7 +421,7 @@ replay_pipe_kernel(const __nv_bfloat16* __restrict__ S_hi, const __nv_bfloat16* 
       __syncwarp();
       if (lane < 8) {                                 // decay products and per-position scalars
         const int pd = 8 * cw + lane;
-        const int io = ps[pd].io, b = ps[pd].b, wnew = ps[pd].wnew;
+        const int b = ps[pd].b, wnew = ps[pd].wnew;
         float al[kPipeMaxT - 1];
 #pragma unroll
         for (int sl = 0; sl < kPipeMaxT - 1; ++sl) {
