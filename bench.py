@@ -67,6 +67,22 @@ def tensor_flops_per_step(w: wl.Workload) -> int:
     return 4 * w.d_v * w.d_k * w.B * w.R * w.H
 
 
+def algorithmic_flops_per_step(w: wl.Workload) -> list:
+    """Floating-point operations the projection replay performs at each decode step t, counted
+    per beam as the method states them (a multiply-add is two): the two shared-state
+    contractions S_ctx q and S_ctx k (4 d_v d_k), the t - 1 ancestors' key products with k and q
+    (4 d_k each) and their accumulation into u and o (4 d_v each), and the new record and the
+    output (8 d_v)."""
+    dk, dv = w.d_k, w.d_v
+    return [w.R * w.H * w.B * (4 * dv * dk + 4 * t * (dk + dv) + 8 * dv) for t in range(w.T)]
+
+
+def fullstate_flops_per_step(w: wl.Workload) -> list:
+    """Floating-point operations of the FullState recurrence per step: per beam S k, the rank-1
+    update alpha (S - beta u k^T) + beta v k^T and S q, 8 d_v d_k."""
+    return [w.R * w.H * w.B * 8 * w.d_v * w.d_k for _ in range(w.T)]
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -636,6 +652,41 @@ def fullstate_bytes_per_step(w: wl.Workload, parents: np.ndarray) -> list:
     return out
 
 
+def sweep_shapes(args):
+    """The sweep's grid (or the subset the --sweep-* options select), as (d_k, d_v, R, B, T)."""
+    geoms = SWEEP_GEOMETRIES if not args.sweep_geometry else \
+        tuple(tuple(int(x) for x in g.split("x")) for g in args.sweep_geometry.split(","))
+    Rs = SWEEP_REQUESTS if not args.sweep_requests else \
+        tuple(int(x) for x in args.sweep_requests.split(","))
+    Bs = SWEEP_BEAMS if not args.sweep_beams else tuple(int(x) for x in args.sweep_beams.split(","))
+    Ts = SWEEP_STEPS if not args.sweep_steps else tuple(int(x) for x in args.sweep_steps.split(","))
+    return [(dk, dv, R, B, T) for dk, dv in geoms for R in Rs for B in Bs for T in Ts]
+
+
+def run_sweep_model(args):
+    """Host-side models of every sweep shape, no GPU: each path's compulsory bytes and FLOPs per
+    decode, their ratio (arithmetic intensity, FLOP per byte) against the machine balance of
+    the measured peaks (dense bf16 tensor FLOP/s over HBM bytes/s), and the capacity bytes. The
+    workloads and parent tables are those the timed sweep uses (same seeds)."""
+    peaks = measured_peaks()
+    balance = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    for dk, dv, R, B, T in sweep_shapes(args):
+        w = wl.Workload(f"sweep_dk{dk}_dv{dv}_R{R}_B{B}_T{T}", R=R, H=16, d_k=dk, d_v=dv,
+                        P=1024, B=B, T=T, parent_law="zipf", zipf_s=1.0, seed=1005)
+        parents = wl.make_parents(w)
+        rb, rf = sum(algorithmic_bytes_per_step(w, parents)), sum(algorithmic_flops_per_step(w))
+        fb, ff = sum(fullstate_bytes_per_step(w, parents)), sum(fullstate_flops_per_step(w))
+        print(json.dumps({
+            "d_k": dk, "d_v": dv, "R": R, "H": w.H, "B": B, "T": T,
+            "replay": {"bytes": int(rb), "flops": int(rf), "flop_per_byte": rf / rb},
+            "fullstate": {"bytes": int(fb), "flops": int(ff), "flop_per_byte": ff / fb},
+            "machine_balance_flop_per_byte": balance,
+            "capacity": {"replay_record_bytes_per_beam_head_step": 4 * dv + w.elem_bytes * dk + 4,
+                         "replay_shared_state_bytes_per_request_head": 4 * dv * dk,
+                         "fullstate_bytes_per_beam_head": 4 * dv * dk}}), flush=True)
+    return 0
+
+
 def run_sweep(args):
     """The operator sweep: nine (d_k, d_v) geometries x request counts x beam widths x decode
     lengths (405 shapes), H = 16 heads, bf16 inputs, Zipf(1.0) parents, a shared state from a
@@ -649,12 +700,11 @@ def run_sweep(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     peaks = measured_peaks()
-    geoms = SWEEP_GEOMETRIES if not args.sweep_geometry else \
-        tuple(tuple(int(x) for x in g.split("x")) for g in args.sweep_geometry.split(","))
-    Rs = SWEEP_REQUESTS if not args.sweep_requests else \
-        tuple(int(x) for x in args.sweep_requests.split(","))
-    Bs = SWEEP_BEAMS if not args.sweep_beams else tuple(int(x) for x in args.sweep_beams.split(","))
-    Ts = SWEEP_STEPS if not args.sweep_steps else tuple(int(x) for x in args.sweep_steps.split(","))
+    shapes = sweep_shapes(args)
+    geoms = tuple(dict.fromkeys((dk, dv) for dk, dv, _, _, _ in shapes))
+    Rs = tuple(dict.fromkeys(R for _, _, R, _, _ in shapes))
+    Bs = tuple(dict.fromkeys(B for _, _, _, B, _ in shapes))
+    Ts = tuple(dict.fromkeys(T for _, _, _, _, T in shapes))
     stream = torch.cuda.current_stream()
 
     def timed(dec, steps, par, outs, reps, warm):
@@ -706,9 +756,11 @@ def run_sweep(args):
                     ms = timed(dec, steps, par, outs, reps, 0)
                     dec.close()
                     rb = sum(algorithmic_bytes_per_step(w, parents))
+                    rf = sum(algorithmic_flops_per_step(w))
                     row["replay"] = {"ms": ms, "beam_head_steps_per_s": bh_steps / (ms / 1e3),
                                      "bytes": int(rb), "gbs": rb / (ms / 1e3) / 1e9,
-                                     "hbm_frac": rb / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+                                     "hbm_frac": rb / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                                     "flops": int(rf), "flop_per_byte": rf / rb}
                     o_rep = [o.clone() for o in outs] if args.sweep_check else None
                     fsb = 2 * R * w.H * B * dv * dk * 4
                     row["capacity"] = {
@@ -724,7 +776,9 @@ def run_sweep(args):
                         fms = timed(dec, steps, par, outs, reps, 0)
                         dec.close()
                         fb = sum(fullstate_bytes_per_step(w, parents))
-                        row["fullstate"] = {"ms": fms, "bytes": int(fb),
+                        ff = sum(fullstate_flops_per_step(w))
+                        row["fullstate"] = {"ms": fms, "bytes": int(fb), "flops": int(ff),
+                                            "flop_per_byte": ff / fb,
                                             "gbs": fb / (fms / 1e3) / 1e9,
                                             "hbm_frac": fb / (fms / 1e3) / 1e9 / peaks["hbm_gbs"],
                                             "replay_speedup": fms / ms}
@@ -771,10 +825,14 @@ def main():
     ap.add_argument("--sweep-check", action="store_true",
                     help="also report the largest |o| difference between replay and FullState")
     ap.add_argument("--sweep-no-fullstate", action="store_true")
+    ap.add_argument("--sweep-model", action="store_true",
+                    help="print the sweep's byte, FLOP and capacity models per shape (no GPU)")
     args = ap.parse_args()
     for name in args.workload.split(","):
         if name not in wl.WORKLOADS:
             ap.error(f"unknown workload {name}")
+    if args.sweep_model:
+        return run_sweep_model(args)
     if args.sweep:
         return run_sweep(args)
     if args.warmup < 3 and args.impl == "ours":

@@ -70,3 +70,15 @@ def test_state_and_record_bytes_are_the_full_bytes_minus_the_io():
         io = w.R * w.H * w.B * ((2 * w.d_k + w.d_v) * e + 8 + 4 * w.d_v)
         rows = w.R * 4 * w.B * (t + 2)
         assert full[t] - lit[t] == io + rows
+
+
+def test_flop_models_per_step():
+    """Replay: the two shared-state contractions plus per-ancestor key products and
+    accumulations, one ancestor more at each step; FullState: a fixed 8 d_v d_k per beam."""
+    w = wl.Workload("t", R=2, H=3, d_k=16, d_v=8, P=1, B=5, T=4, parent_law="uniform")
+    rep = bench.algorithmic_flops_per_step(w)
+    n = w.R * w.H * w.B
+    assert rep[0] == n * (4 * w.d_v * w.d_k + 8 * w.d_v)
+    assert all(rep[t + 1] - rep[t] == n * 4 * (w.d_k + w.d_v) for t in range(w.T - 1))
+    assert rep[0] - n * 8 * w.d_v == bench.tensor_flops_per_step(w)
+    assert bench.fullstate_flops_per_step(w) == [n * 8 * w.d_v * w.d_k] * w.T
