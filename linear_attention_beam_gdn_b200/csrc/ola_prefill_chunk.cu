@@ -23,7 +23,7 @@
 //              its key tile has landed
 //   warp 15    tcgen05.mma: N of each chunk once its M2 tiles are written
 //   warps 0-3, 10-13  two precompute groups taking alternate chunks, ahead of the state chain:
-//              gates (prefix sums, beta D, -a_C beta), L = diag(beta) K~ from the Gram matrix,
+//              gates (prefix sums, beta, beta D, -a), L = diag(beta) K~ from the Gram matrix,
 //              T = (I + L)^-1 in fp32 by 16 x 16 blocks (diagonal blocks by forward
 //              substitution, the others by block products over two halves of 32),
 //              M1 and M2 as bf16 hi + lo tiles
